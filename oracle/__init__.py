@@ -1,0 +1,9 @@
+"""CPU oracle for the BitSSM forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute anything in this package: only ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` use it.  It shares no code with the
+CUDA library and imports nothing from it.
+"""
+
+from .bitssm_oracle import *  # noqa: F401,F403
