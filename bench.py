@@ -1,0 +1,457 @@
+"""Benchmark of the BitSSM mixer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload trissm]
+
+One step = one bitssm_forward (every stage of the mixer: quantise x, in_proj,
+x_proj, the selective scan with Delta-up fused, quantise y, out_proj, plus the
+per-call weight expansion) over one batch of the workload.  Rank 0 prints one
+JSON line.
+
+Timing: W untimed warm-up steps, then K timed steps between a barrier and a
+device synchronise on both sides.  The workload's working set fits in the
+126 MB L2, so before every timed step a 256 MiB buffer is overwritten (L2
+flush) and each step is timed alone with CUDA events on the launching stream
+(the flush is outside the events).  Multi-GPU: one process per GPU, each
+runs its own batch (weak scaling, no collective on the data path); the
+reported time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the plain float64 reference of the
+method) on the same workload, on a bounded sample per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "BitSSM mixer tokens/s on 1 B200; % of int8-TC / HBM roofline"
+UNIT = "tokens/s"
+MUFU_EX2_PER_CLK_PER_SM = 16      # special-function unit exp2 rate per SM per clock
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": SM_MAX_MHZ}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        mhz, max_mhz, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                max_mhz = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- byte counts
+
+def scan_bytes_per_token(E, N, R_pad):
+    """Algorithmic bytes of the fused scan kernel per token: read u (fp32),
+    the Delta-down codes and their factor, B and C (fp32); write y (fp32)."""
+    return E * 4 + R_pad + 4 + 2 * N * 4 + E * 4
+
+
+def layer_bytes_per_token(wl):
+    """Algorithmic HBM bytes of the whole unfused A8 forward per token (each
+    kernel reads its inputs and writes its outputs once)."""
+    d, E, N = wl.d_model, wl.d_inner, wl.d_state
+    Rp = (wl.dt_rank + 15) // 16 * 16
+    io = 2 if wl.io_dtype == "bf16" else 4
+    quant_x = d * io + d + 4
+    in_proj = d + 4 + E * 4 + E + 4
+    x_proj = E + 4 + 2 * N * 4 + Rp + 4
+    scan = scan_bytes_per_token(E, N, Rp)
+    quant_y = E * 4 + E + 4
+    out_proj = E + 4 + d * io
+    return quant_x + in_proj + x_proj + scan + quant_y + out_proj
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from ternary_weight_selective_b200 import bitssm as abi
+    from ternary_weight_selective_b200 import device as dev
+    from ternary_weight_selective_b200 import synthetic as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    wl = S.WORKLOADS[args.workload]
+    act = abi.A16 if wl.act_mode == "A16" else abi.A8
+    dtype = abi.BF16 if wl.io_dtype == "bf16" else abi.F32
+    B, L = wl.batch, wl.seqlen
+    T = B * L
+    x, layers = S.make_inputs(wl, seed=rank)
+    dl = [dev.DeviceLayer(lw, act) for lw in layers]
+    stream = torch.cuda.current_stream()
+    xd = dev.to_device_input(x, dtype)
+    out = torch.empty_like(xd)
+    nbytes = abi.bitssm_workspace_size(dl[0].layer, B, L, dtype, act)
+    ws = dev.Workspace(nbytes)
+    nl = abi.bitssm_forward_launches(dl[0].layer, act)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record()  # creates the underlying cudaEvent_t
+        return evs
+
+    n_layers = len(dl)
+    per_step = n_layers * (nl + 1)
+
+    def step(evs):
+        """One forward; evs: (nl + 1) events per layer, recorded by the library
+        before every kernel and after the last."""
+        st = torch.cuda.current_stream()
+        h_in = xd
+        for li, d_l in enumerate(dl):
+            e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
+            abi.bitssm_forward_timed(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B, L,
+                                     dtype, act, ws.addr, nbytes, [ev.cuda_event for ev in e], st)
+            h_in = out
+
+    # eager warm-up (also sets the kernels' shared-memory attributes)
+    warm = new_events(per_step)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(warm)
+    torch.cuda.synchronize()
+
+    # The timed steps run as CUDA-graph replays (host launch cost out of the
+    # device timeline): one graph holds G x (L2 flush + timed forward).
+    G = max(1, min(args.steps, 100))
+    R = (args.steps + G - 1) // G
+    K = G * R
+    gevents = [new_events(per_step) for _ in range(G)]
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cap):
+        for i in range(G):
+            flush.zero_()
+            step(gevents[i])
+    torch.cuda.synchronize()
+    graph.replay()  # one untimed replay
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(local)
+    gpu_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    sampler = ClockSampler(gpu_id)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    step_ms, kern_ms = [], [[0.0] * nl for _ in range(n_layers)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for r in range(R):
+        graph.replay()
+        torch.cuda.synchronize()
+        for evs in gevents:
+            tot = 0.0
+            for li in range(n_layers):
+                e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
+                for i in range(nl):
+                    kern_ms[li][i] += e[i].elapsed_time(e[i + 1])
+                tot += e[0].elapsed_time(e[nl])
+            step_ms.append(tot)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    del graph
+    args.steps = K
+
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = T * world / (ms_per_step / 1e3)
+
+    # ---------------- end to end through the C ABI with host buffers
+    x_host = torch.empty(xd.shape, dtype=xd.dtype, pin_memory=True)
+    x_host.copy_(xd.cpu())
+    out_host = torch.empty(xd.shape, dtype=xd.dtype, pin_memory=True)
+    x_dev2 = torch.empty_like(xd)
+    n_e2e = min(args.steps, 200)
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_e2e)]
+
+    def e2e_step():
+        x_dev2.copy_(x_host, non_blocking=True)
+        h_in = x_dev2
+        for d_l in dl:
+            abi.bitssm_forward(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B, L, dtype,
+                               act, ws.addr, nbytes, torch.cuda.current_stream())
+            h_in = out
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for k in range(n_e2e):
+        flush.zero_()
+        e0[2 * k].record()
+        e2e_step()
+        e0[2 * k + 1].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(e0[2 * k].elapsed_time(e0[2 * k + 1]) for k in range(n_e2e))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = T * world / (e2e_ms / n_e2e / 1e3)
+    io_bytes = T * wl.d_model * (2 if dtype == abi.BF16 else 4)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    # ---------------- roofline of the dominant kernel
+    names_a8 = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_x_proj",
+                "selective_scan_fused_dt", "quant_rows_y", "gemm_out_proj"]
+    names = names_a8 if act == abi.A8 else ["expand_weights", "row_rms_x", "gemm_in_proj",
+                                            "gemm_x_proj", "gemm_dt_proj", "selective_scan",
+                                            "row_rms_y", "gemm_out_proj"]
+    if nl == len(names) - 1:
+        names = names[1:]
+    avg_kernel_ms = [sum(kern_ms[li][i] for li in range(n_layers)) / (args.steps * n_layers)
+                     for i in range(nl)]
+    share = {names[i]: round(avg_kernel_ms[i] / (ms_per_step / n_layers), 4) for i in range(nl)}
+    dom = max(range(nl), key=lambda i: avg_kernel_ms[i])
+    peaks, peak_kind = load_peaks()
+    sm_max = (clocks or {}).get("sm_max_mhz") or peaks.get("sm_max_mhz", SM_MAX_MHZ)
+    Rp = (wl.dt_rank + 15) // 16 * 16
+    roof = None
+    if names[dom].startswith("selective_scan"):
+        exps = T * wl.d_inner * wl.d_state
+        t_s = avg_kernel_ms[dom] / 1e3
+        achieved = exps / t_s / 1e12
+        peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e12
+        hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp)
+        roof = {"kernel": names[dom], "bound": "alu", "unit": "Tex2/s",
+                "achieved": round(achieved, 4), "peak": round(peak, 4),
+                "frac": round(achieved / peak, 4),
+                "peak_source": f"{MUFU_EX2_PER_CLK_PER_SM} ex2/clk/SM x {SM_COUNT} SMs x {sm_max:.0f} MHz",
+                "traffic": None,
+                "hbm_achieved_gbs": round(hbm_bytes / t_s / 1e9, 1),
+                "hbm_frac": round(hbm_bytes / t_s / 1e9 / peaks["hbm_gbs"], 4),
+                "hbm_peak_source": f"{peak_kind} hbm_gbs"}
+    else:
+        t_s = avg_kernel_ms[dom] / 1e3
+        bytes_all = T * layer_bytes_per_token(wl)
+        roof = {"kernel": names[dom], "bound": "hbm", "unit": "GB/s",
+                "achieved": round(bytes_all / t_s / 1e9, 1), "peak": peaks["hbm_gbs"],
+                "frac": None, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs"}
+    layer_gbs = T * layer_bytes_per_token(wl) / (ms_per_step / n_layers / 1e3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8/int32 (A8) with fp32 scan" if act == abi.A8 else "bf16/fp32 (A16)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "seq_len": L, "d_model": wl.d_model,
+                   "d_inner": wl.d_inner, "d_state": wl.d_state, "dt_rank": wl.dt_rank,
+                   "layers": n_layers, "io_dtype": wl.io_dtype, "act_mode": wl.act_mode,
+                   "parallelism": f"replica x{world}" if world > 1 else "single",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+        "roofline": roof,
+        "kernel_share": share,
+        "kernel_avg_us": {names[i]: round(avg_kernel_ms[i] * 1e3, 2) for i in range(nl)},
+        "layer_hbm_gbs_algorithmic": round(layer_gbs, 1),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
+                "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": args.steps * n_layers * nl,
+        "clocks": clocks,
+        "wall_s_timed_region": round(t_wall, 4),
+        "timing": f"{R} replays of a CUDA graph of {G} x (L2 flush + forward); per-kernel CUDA events inside the graph",
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------- oracle arms
+
+def _oracle_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        return max(blas) if blas else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl, seqs: int):
+    from oracle import bitssm_oracle as O
+    from ternary_weight_selective_b200 import synthetic as S
+    x, layers = S.make_inputs(wl, seed=0, batch=seqs)
+    P = [O.TernaryLayer(lw, wl.act_mode) for lw in layers]
+
+    def run():
+        if len(P) == 1:
+            O.bitssm_layer(x, P[0])
+        else:
+            O.bitssm_stack(x, P)
+    return run, seqs * wl.seqlen
+
+
+def cpu_baseline(wl, budget_s: float = 12.0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    sequences of the workload's length, repeated until ~budget_s of CPU work."""
+    seqs = max(1, min(wl.batch, 4))
+    run, tokens = oracle_sample(wl, seqs)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        run()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 50:
+            break
+    return {"value": round(tokens * n / el, 1), "unit": UNIT, "cores": _oracle_threads(),
+            "kind": "oracle", "sample": f"{n} x {seqs} sequences x {wl.seqlen} tokens "
+                                        f"({wl.layers} layer(s)), {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from ternary_weight_selective_b200 import synthetic as S
+    wl = S.WORKLOADS[args.workload]
+    seqs = max(1, min(wl.batch, 2))
+    run, tokens = oracle_sample(wl, seqs)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    value = tokens * args.steps / el
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (int codes decided in f32)", "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen,
+                   "d_model": wl.d_model, "d_inner": wl.d_inner, "d_state": wl.d_state,
+                   "dt_rank": wl.dt_rank, "layers": wl.layers, "io_dtype": wl.io_dtype,
+                   "act_mode": wl.act_mode, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": _oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: {seqs} sequences x {wl.seqlen} tokens"},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="trissm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

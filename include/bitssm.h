@@ -1,0 +1,263 @@
+/*
+ * bitssm.h - C ABI of the BitSSM forward library for NVIDIA B200 (sm_100a).
+ *
+ * BitSSM is the selective state-space sequence mixer of TriSSM whose
+ * projections are BitNet b1.58 BitLinear layers: ternary {-1, 0, +1} weights
+ * and int8 activations ("Associative Recall Under Ternary Quantization: A
+ * Controlled Comparison of State Space Models and Transformers at 5M
+ * Parameters", TriSSM repository README: opening paragraph, the caption "The
+ * BitSSM sequence mixer", the Overview table and "Repository structure").
+ * The W1.58A16 variant (16-bit activations, grouped weight scales) follows
+ * "Ternary Mamba: Grouped Quantization-Aware Training of W1.58A16 State
+ * Space Models" (abstract).
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor arguments are DEVICE pointers owned by the caller, row-major and
+ *    densely packed unless a leading dimension is stated.  Structs
+ *    (bitssm_tw, bitssm_layer) are HOST memory; their pointer fields are
+ *    device pointers.  The library keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work on that stream and return without
+ *    synchronising; results are ready when the stream reaches them.
+ *  - The forward entry points allocate no device memory: scratch comes from
+ *    the caller's workspace `ws` of `ws_bytes` bytes (256-byte aligned),
+ *    sized by the matching *_workspace_size query.
+ *  - Return value: BITSSM_OK, or an error status.  Argument errors are
+ *    detected on the host before anything is enqueued.  BITSSM_ERR_CUDA
+ *    reports a launch error.  Device-side conditions (a bounded wait that ran
+ *    out) are recorded in a device error word read by bitssm_device_error().
+ *  - Element types: BITSSM_F32 (float), BITSSM_BF16 (bfloat16 bits),
+ *    BITSSM_I32 (int32, only as a raw-accumulator output).
+ *  - The library computes on the current CUDA device; pointers must belong
+ *    to it.
+ */
+#ifndef BITSSM_H
+#define BITSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BITSSM_ABI_VERSION 1
+
+enum bitssm_status_code {
+  BITSSM_OK = 0,
+  BITSSM_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad enum */
+  BITSSM_ERR_UNSUPPORTED_SHAPE = 2,/* a size this build does not support */
+  BITSSM_ERR_WORKSPACE = 3,        /* workspace missing, misaligned or too small */
+  BITSSM_ERR_CUDA = 4,             /* a CUDA launch or runtime call failed */
+  BITSSM_ERR_TIMEOUT = 5,          /* a bounded device wait ran out (device error word) */
+  BITSSM_ERR_DEVICE_FLAG = 6       /* another device-side check failed */
+};
+
+enum bitssm_dtype { BITSSM_F32 = 0, BITSSM_BF16 = 1, BITSSM_I32 = 2 };
+
+/* Activation modes.  A8: per-token absmax int8 activation codes (BitNet
+ * b1.58; TriSSM README opening paragraph).  A16: bf16 activations without
+ * activation quantisation, weights with per-group scales (W1.58A16; Ternary
+ * Mamba abstract). */
+enum bitssm_act_mode { BITSSM_A8 = 0, BITSSM_A16 = 1 };
+
+/* Ternary weight matrix W_q [n_out, k_in] in the 2-bit encoding:
+ *   packed: uint8 [n_out, ceil(k_in/4)]; element (n, k) is the code
+ *           c = w + 1 in {0, 1, 2} at bits 2*(k mod 4) of byte k/4 of row n;
+ *           code 3 is invalid; padding elements hold c = 1 (w = 0).
+ *   scales: float absmean scales; group == 0: one float (per matrix);
+ *           group == 128: float [n_out, ceil(k_in/128)], scale of each run
+ *           of 128 consecutive k of one row.
+ * A8 layers use group 0; A16 layers use group 128. */
+typedef struct bitssm_tw {
+  const uint8_t* packed;
+  const float* scales;
+  int n_out;
+  int k_in;
+  int group;
+} bitssm_tw;
+
+/* Weights of one BitSSM mixer.  Shapes (d = d_model, E = d_inner,
+ * N = d_state, R = dt_rank):
+ *   in_proj  [E, d]    dt_down [R, E]   b_proj [N, E]   c_proj [N, E]
+ *   dt_up    [E, R]    out_proj [d, E]
+ *   A [E, N] float (the negative decay rates), D [E] float (skip),
+ *   dt_bias [E] float (added before the softplus).
+ * `prepared` may point to a device buffer filled by bitssm_prepare_weights()
+ * for this layer and act mode (the weights expanded to tensor-core operand
+ * form), or be NULL: the forward then expands them into its workspace on
+ * every call. */
+typedef struct bitssm_layer {
+  bitssm_tw in_proj, dt_down, b_proj, c_proj, dt_up, out_proj;
+  const float* A;
+  const float* D;
+  const float* dt_bias;
+  int d_model;
+  int d_inner;
+  int d_state;
+  int dt_rank;
+  const void* prepared;
+} bitssm_layer;
+
+/* Version of this ABI (BITSSM_ABI_VERSION). */
+int bitssm_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* bitssm_status_string(int status);
+
+/* Name and description of the last CUDA error a call of this library saw on
+ * the calling thread (behind a BITSSM_ERR_CUDA status); "no error" before
+ * any.  The string stays valid until the thread's next failing call. */
+const char* bitssm_last_error(void);
+
+/* Reads the device error word of the current device into *flags (bit 0: a
+ * TMA wait ran out, bit 1: an MMA-completion wait ran out, bit 2: an
+ * epilogue wait ran out) after synchronising the device; clears it when
+ * `clear` is non-zero.  Returns BITSSM_OK, or BITSSM_ERR_TIMEOUT when any
+ * bit was set, or BITSSM_ERR_CUDA. */
+int bitssm_device_error(unsigned int* flags, int clear);
+
+/* ---------------------------------------------------------------------
+ * Weight packing (offline).  Absmean ternarisation of the BitNet b1.58
+ * BitLinear (TriSSM README opening paragraph; grouped scales: Ternary Mamba
+ * abstract):
+ *   s = mean |W| over the matrix (group 0) or over each run of `group`
+ *       consecutive k of a row (group 128), summed in float64, stored as
+ *       float;
+ *   W_q = clip(rint(W / (s + 1e-5)), -1, 1), the division in float32,
+ *       rint = round half to even.
+ * W: float [n_out, k_in] device.  packed: uint8 [n_out, ceil(k_in/4)]
+ * (every byte written).  scales: 1 float (group 0) or
+ * [n_out, ceil(k_in/group)] floats.  ws: bitssm_pack_workspace_size bytes.
+ * --------------------------------------------------------------------- */
+int bitssm_pack_workspace_size(int n_out, int k_in, int group, size_t* bytes);
+int bitssm_pack_ternary(const float* W, int n_out, int k_in, int group, uint8_t* packed,
+                        float* scales, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------
+ * BitLinear forward on M input rows (TriSSM README: opening paragraph and
+ * the caption "an RMSNorm precedes each ternary projection"; multiply-free
+ * ternary GEMM: "Ternary State-Space Models" abstract).
+ *
+ * A8: for each row v of x [M, k_in]: m = max|v|; codes
+ *     q = clamp(rint(v * (127/m)), -128, 127) decided in float32 (all-zero
+ *     codes when m = 0); acc = q W_q^T accumulated exactly in int32 on the
+ *     tensor cores; r = 1/sqrt(mean(v^2) + 1e-5) (unit-gain RMSNorm folded
+ *     into the quantiser); y = acc * s * m * r / 127.
+ *     x_dtype: BITSSM_F32 or BITSSM_BF16.  y_dtype: F32, BF16, or I32 to
+ *     receive the raw int32 accumulators acc.
+ * A16: x bf16 [M, k_in] (k_in a multiple of 8), no activation codes:
+ *     y = r * sum_j s[n, j] * sum_{k in group j} W_q[n, k] * x[k]; the group
+ *     scale enters the bf16 tensor-core operand as bf16(s), so y carries a
+ *     relative error of at most 2^-9 per group from that rounding.
+ *     y_dtype: F32 or BF16.
+ * y: [M, n_out].  ws: bitlinear_workspace_size bytes.
+ * --------------------------------------------------------------------- */
+int bitlinear_workspace_size(const bitssm_tw* w, int M, int act_mode, size_t* bytes);
+int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, void* y, int y_dtype,
+                      int act_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Selective scan (the BitSSM recurrence; TriSSM README caption and
+ * "Repository structure": the recurrence is evaluated with a parallel
+ * associative scan).  For every batch b, channel e, state n, step t:
+ *   delta = softplus(delta_raw[b,t,e] + delta_bias[e])
+ *   h[b,e,n] = exp(delta * A[e,n]) * h[b,e,n] + delta * Bm[b,t,n] * u[b,t,e]
+ *   y[b,t,e] = sum_n Cm[b,t,n] * h[b,e,n] + D[e] * u[b,t,e]
+ * with h = h0 (or 0 when h0 is NULL) before step 0; h_last (nullable)
+ * receives h after step L-1.  Arithmetic in float32.
+ * u, delta_raw, y: [B, L, E] of `dtype` (F32 or BF16); Bm, Cm: float
+ * [B, L, N]; A: float [E, N]; D, delta_bias: float [E]; h0, h_last: float
+ * [B, E, N].  Supported: N = 16, E a multiple of 8, L >= 1.
+ * --------------------------------------------------------------------- */
+int selective_scan_forward(const void* u, const void* delta_raw, const float* delta_bias,
+                           const float* A, const float* Bm, const float* Cm, const float* D,
+                           const float* h0, void* y, float* h_last, int B, int L, int E, int N,
+                           int dtype, void* stream);
+
+/* ---------------------------------------------------------------------
+ * BitSSM mixer forward (one layer): x [B, L, d_model] of `dtype` (F32 or
+ * BF16) -> out [B, L, d_model] of the same dtype; with `residual`
+ * (nullable, same shape and dtype) out = residual + mixer(x).
+ *
+ * A8 (TriSSM form):
+ *   u      = BitLinear_in(x)                              [B,L,E]
+ *   dt_low = BitLinear_dt_down(u), Bm = BitLinear_B(u), Cm = BitLinear_C(u),
+ *            sharing one RMSNorm + quantisation of u, each with its own s
+ *   delta  = softplus(BitLinear_dt_up(dt_low) + dt_bias)
+ *   y      = selective scan of (u, delta, A, Bm, Cm, D), h0 = 0
+ *   out    = BitLinear_out(y)
+ *   The codes fed to dt_down/B/C and to dt_up are decided on the int32
+ *   accumulator rows of the projection before them (in real arithmetic the
+ *   same codes as those of the rescaled rows; exact in float32 because
+ *   |acc| < 2^24).
+ * A16 (W1.58A16 form): the same graph with every BitLinear in A16 form.
+ * Requirements: d_state == 16; d_model and d_inner multiples of 16;
+ * A8: d_inner <= 512; A16: d_model, d_inner multiples of 64.
+ * ws: bitssm_workspace_size bytes.
+ * --------------------------------------------------------------------- */
+int bitssm_workspace_size(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
+                          size_t* bytes);
+int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* residual, int B,
+                   int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernels one bitssm_forward call launches for this layer and act
+ * mode (A8: 6, A16: 7, plus 1 for the weight expansion when `prepared` is
+ * NULL), or -1 for a bad argument.  A8 launch order: [expand] quantise x,
+ * in_proj, x_proj, scan (with Delta-up fused), quantise y, out_proj.  A16:
+ * [expand] RMS of x, in_proj, x_proj, dt_proj, scan, RMS of y, out_proj. */
+int bitssm_forward_launches(const bitssm_layer* p, int act_mode);
+
+/* bitssm_forward, additionally recording events[i] (cudaEvent_t handles
+ * created by the caller, passed as void*) on `stream` before the i-th kernel
+ * and events[n] after the last of the n = bitssm_forward_launches() kernels,
+ * for per-kernel timing.  n_events must be at least n + 1.  Same results and
+ * errors as bitssm_forward. */
+int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const void* residual,
+                         int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* const* events, int n_events, void* stream);
+
+/* Residual stack (TriSSM README Overview table: 12 layers at d = 256):
+ * out = x; for each layer l: out = out + mixer_l(out), rounded to `dtype`.
+ * `layers` is a host array of n_layers layer structs of identical shapes.
+ * ws: bitssm_workspace_size bytes of one layer. */
+int bitssm_stack_forward(const bitssm_layer* layers, int n_layers, const void* x, void* out,
+                         int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Expanded weights: the six ternary matrices of a layer expanded once to
+ * tensor-core operand form (A8: int8 {-1,0,1}; A16: bf16 w * bf16(s)).
+ * bitssm_prepare_weights fills `dst` (bitssm_prepared_size bytes, device,
+ * 256-byte aligned); a layer whose `prepared` field points to it skips the
+ * per-call expansion.  The buffer stays valid while the packed weights do
+ * not change. */
+int bitssm_prepared_size(const bitssm_layer* p, int act_mode, size_t* bytes);
+int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_t dst_bytes,
+                           void* stream);
+
+/* Inspection of the forward's intermediates inside a workspace (for
+ * stage-by-stage checks).  Fills byte offsets into the workspace, or
+ * (size_t)-1 for a buffer the act mode does not use, and the row pitch in
+ * elements of each buffer.
+ *   A8:  q_x int8 [T, ld_qx], deq_x float [T], u float [T, E],
+ *        q_u int8 [T, ld_qu], deq_u float [T], Bm float [T, N],
+ *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],
+ *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]
+ *   A16: r_x float [T], u bf16 [T, E], dt_low bf16 [T, R], r_dt float [T],
+ *        Bm, Cm float [T, N], delta_raw float [T, E], y bf16 [T, E],
+ *        r_y float [T]
+ * deq_* is the per-token factor m * r / 127 of the absmax codes; r_* the
+ * RMSNorm factor. */
+typedef struct bitssm_ws_view {
+  size_t q_x, deq_x, u, q_u, deq_u, Bm, Cm, q_dt, deq_dt, y, q_y, deq_y;
+  size_t r_x, dt_low, r_dt, delta_raw, r_y;
+  int ld_qx, ld_qu, ld_qdt;
+} bitssm_ws_view;
+int bitssm_workspace_layout(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
+                            bitssm_ws_view* view);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITSSM_H */

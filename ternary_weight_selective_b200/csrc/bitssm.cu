@@ -1,0 +1,841 @@
+// C ABI of the BitSSM forward library (declarations and contracts in
+// include/bitssm.h): argument checks, the workspace plan, TMA descriptor
+// encoding, and the launch sequence of each entry point.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "bitssm.h"
+#include "kernel_gemm.cuh"
+#include "kernel_scan.cuh"
+#include "kernels_rows.cuh"
+#include "ptx.cuh"
+
+namespace bitssm {
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Name of the last CUDA error this library saw on this thread.
+thread_local char g_last_error[160] = "no error";
+void note_cuda_error(cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+}
+// Status of the launches enqueued since the previous check.
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return BITSSM_OK;
+  note_cuda_error(e);
+  return BITSSM_ERR_CUDA;
+}
+
+int g_num_sms = 0;
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D K-major operand [rows, k] with row pitch `ld` elements; box = one
+// 128-byte K panel x box_rows rows, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* map, const void* ptr, bool bf16, long k, long rows, long ld,
+              int box_rows) {
+  if (!get_encode()) return false;
+  const int esz = bf16 ? 2 : 1;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) != 0 || (ld * esz) % 16 != 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                        2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ GEMM launch
+template <bool kBF16, int BN, int EPI>
+int launch_gemm_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
+                   const GemmParams& P, cudaStream_t st) {
+  constexpr int kStage = 128 * 128 + BN * 128;
+  constexpr int kStages = (200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage);
+  using Cfg = GemmConfig<kBF16, BN, kStages, EPI>;
+  auto kern = ternary_gemm_kernel<kBF16, BN, kStages, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return BITSSM_ERR_CUDA;
+    attr_set = true;
+  }
+  CUtensorMap mA, mW;
+  if (!make_map(&mA, A, kBF16, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (!make_map(&mW, W, kBF16, P.K, w_rows, ldw, BN > 256 ? 256 : BN))
+    return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  dim3 grid((P.M + 127) / 128, (P.N + BN - 1) / BN);
+  kern<<<grid, 192, Cfg::kSmemBytes, st>>>(mA, mW, P);
+  return launch_status();
+}
+
+// N-tile choice: the smallest instantiated BN covering the columns the
+// epilogue needs in one tile (whole-row epilogues), else 256 with N tiling.
+template <bool kBF16, int EPI>
+int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, const GemmParams& P,
+                cudaStream_t st) {
+  const int need = (EPI == EPI_STORE || EPI == EPI_ROWSS) ? (P.N < 256 ? P.N : 256) : P.N;
+  if (need <= 64) return launch_gemm_bn<kBF16, 64, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if (need <= 128) return launch_gemm_bn<kBF16, 128, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if (need <= 256) return launch_gemm_bn<kBF16, 256, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if constexpr (EPI == EPI_QUANT_ROW) {
+    if (need <= 512) return launch_gemm_bn<kBF16, 512, EPI>(A, lda, W, ldw, w_rows, P, st);
+  }
+  return BITSSM_ERR_UNSUPPORTED_SHAPE;
+}
+
+// N-tile width used by the A16 in_proj (its partial sums are per tile)
+inline int rowss_bn(int N) { return N <= 64 ? 64 : N <= 128 ? 128 : 256; }
+
+// ------------------------------------------------------------ row kernels
+inline int rows_grid(long M) {
+  long g = (M + 7) / 8;
+  long cap = (long)num_sms() * 16;
+  return (int)(g < cap ? (g < 1 ? 1 : g) : cap);
+}
+
+int launch_quant_rows(const void* x, int dtype, int M, int K, long ldx, int8_t* q, long ldq,
+                      float* deq, cudaStream_t st) {
+  if (M == 0) return BITSSM_OK;
+  if (dtype == BITSSM_F32)
+    quant_rows_kernel<float><<<rows_grid(M), 256, 0, st>>>(reinterpret_cast<const float*>(x), M, K,
+                                                           ldx, q, ldq, deq);
+  else
+    quant_rows_kernel<__nv_bfloat16><<<rows_grid(M), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), M, K, ldx, q, ldq, deq);
+  return launch_status();
+}
+
+int launch_row_rms(const void* x, int dtype, int M, int K, long ldx, float* r, cudaStream_t st) {
+  if (M == 0) return BITSSM_OK;
+  if (dtype == BITSSM_F32)
+    row_rms_kernel<float><<<rows_grid(M), 256, 0, st>>>(reinterpret_cast<const float*>(x), M, K,
+                                                        ldx, r);
+  else
+    row_rms_kernel<__nv_bfloat16><<<rows_grid(M), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), M, K, ldx, r);
+  return launch_status();
+}
+
+int launch_expand(const ExpandJobs& jobs, bool bf16, cudaStream_t st) {
+  long total = 0;
+  for (int i = 0; i < jobs.count; ++i)
+    total += (long)jobs.job[i].n_out * (jobs.job[i].ld / (bf16 ? 8 : 16));
+  long g = (total + 255) / 256;
+  long cap = (long)num_sms() * 8;
+  int grid = (int)(g < 1 ? 1 : (g < cap ? g : cap));
+  if (bf16) expand_bf16_kernel<<<grid, 256, 0, st>>>(jobs);
+  else expand_i8_kernel<<<grid, 256, 0, st>>>(jobs);
+  return launch_status();
+}
+
+// ------------------------------------------------------------ scan launch
+template <int NPT, bool FUSED, typename Tu, typename Td, typename Ty>
+int launch_scan_t(const ScanParams& P, cudaStream_t st) {
+  constexpr int CE = 128 * NPT / kScanN;
+  const int Rm = FUSED ? P.R : 0;
+  const int smem = scan_smem_bytes(CE, Rm);
+  auto kern = selective_scan_kernel<NPT, FUSED, Tu, Td, Ty>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return BITSSM_ERR_CUDA;
+  }
+  dim3 grid((P.E + CE - 1) / CE, P.B);
+  kern<<<grid, 128, smem, st>>>(P);
+  return launch_status();
+}
+
+// states per thread: enough threads to fill the machine when B*E is small
+template <bool FUSED, typename Tu, typename Td, typename Ty>
+int launch_scan(const ScanParams& P, cudaStream_t st) {
+  const long channels = (long)P.B * P.E;
+  const long want = (long)num_sms() * 4 * 32 * 6;  // ~6 warps per SM sub-partition
+  if (channels * 16 / 16 >= want) return launch_scan_t<16, FUSED, Tu, Td, Ty>(P, st);
+  if (channels * 16 / 4 >= want) return launch_scan_t<4, FUSED, Tu, Td, Ty>(P, st);
+  return launch_scan_t<1, FUSED, Tu, Td, Ty>(P, st);
+}
+
+// ------------------------------------------------------------ validation
+bool tw_ok(const bitssm_tw* w) {
+  return w != nullptr && w->packed != nullptr && w->scales != nullptr && w->n_out > 0 &&
+         w->k_in > 0 && (w->group == 0 || w->group == 128);
+}
+
+// ------------------------------------------------------------ layer plan
+struct LayerPlan {
+  int T, d, E, N, R;
+  int ld_d, ld_E, ld_R;    // padded K pitches (elements)
+  int xrows;               // R + 2N
+  bool a16;
+  // expanded weights (offsets relative to the expanded block)
+  size_t w_in, w_x, w_up, w_out, w_bytes;
+  // workspace offsets (absolute; expanded block at 0 when not prepared)
+  size_t base;
+  bitssm_ws_view v;
+  size_t ss_u;             // A16 partial sums
+  int ss_parts;
+  size_t total;
+};
+
+bool layer_shape_ok(const bitssm_layer* p, int act_mode) {
+  if (p == nullptr) return false;
+  const bitssm_tw* ws[6] = {&p->in_proj, &p->dt_down, &p->b_proj, &p->c_proj, &p->dt_up, &p->out_proj};
+  for (auto w : ws)
+    if (!tw_ok(w)) return false;
+  if (p->A == nullptr || p->D == nullptr || p->dt_bias == nullptr) return false;
+  const int d = p->d_model, E = p->d_inner, N = p->d_state, R = p->dt_rank;
+  if (d <= 0 || E <= 0 || N <= 0 || R <= 0) return false;
+  if (p->in_proj.n_out != E || p->in_proj.k_in != d) return false;
+  if (p->dt_down.n_out != R || p->dt_down.k_in != E) return false;
+  if (p->b_proj.n_out != N || p->b_proj.k_in != E) return false;
+  if (p->c_proj.n_out != N || p->c_proj.k_in != E) return false;
+  if (p->dt_up.n_out != E || p->dt_up.k_in != R) return false;
+  if (p->out_proj.n_out != d || p->out_proj.k_in != E) return false;
+  const int want_group = act_mode == BITSSM_A16 ? -1 : 0;
+  for (auto w : ws)
+    if (want_group == 0 && w->group != 0) return false;
+  return true;
+}
+
+int layer_supported(const bitssm_layer* p, int act_mode) {
+  if (p->d_state != kScanN) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (p->d_model % 16 != 0 || p->d_inner % 16 != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (act_mode == BITSSM_A8) {
+    if (p->d_inner > 512) return BITSSM_ERR_UNSUPPORTED_SHAPE;   // whole u row in one tile
+    if (p->dt_rank + 2 * p->d_state > 256) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+    if (round_up(p->dt_rank, 16) > 128) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  } else {
+    if (p->dt_rank % 8 != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;  // bf16 TMA pitch
+    if (p->dt_rank + 2 * p->d_state > 256) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  }
+  return BITSSM_OK;
+}
+
+LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool prepared) {
+  LayerPlan P;
+  std::memset(&P, 0, sizeof(P));
+  P.T = B * L;
+  P.d = p->d_model;
+  P.E = p->d_inner;
+  P.N = p->d_state;
+  P.R = p->dt_rank;
+  P.a16 = act_mode == BITSSM_A16;
+  P.ld_d = round_up(P.d, 16);
+  P.ld_E = round_up(P.E, 16);
+  P.ld_R = round_up(P.R, 16);
+  P.xrows = P.R + 2 * P.N;
+  const size_t es = P.a16 ? 2 : 1;
+  size_t o = 0;
+  P.w_in = o; o = align_up(o + (size_t)P.E * P.ld_d * es);
+  P.w_x = o; o = align_up(o + (size_t)P.xrows * P.ld_E * es);
+  P.w_up = o; o = align_up(o + (size_t)P.E * P.ld_R * es);
+  P.w_out = o; o = align_up(o + (size_t)P.d * P.ld_E * es);
+  P.w_bytes = o;
+  size_t a = prepared ? 0 : P.w_bytes;
+  const size_t T = (size_t)P.T;
+  const size_t none = (size_t)-1;
+  bitssm_ws_view& v = P.v;
+  v.q_x = v.deq_x = v.u = v.q_u = v.deq_u = v.Bm = v.Cm = v.q_dt = v.deq_dt = v.y = v.q_y = v.deq_y = none;
+  v.r_x = v.dt_low = v.r_dt = v.delta_raw = v.r_y = none;
+  P.ss_u = none;
+  auto take = [&](size_t bytes) {
+    size_t r = a;
+    a = align_up(a + bytes);
+    return r;
+  };
+  v.ld_qx = P.ld_d;
+  v.ld_qu = P.ld_E;
+  v.ld_qdt = P.ld_R;
+  if (!P.a16) {
+    v.q_x = take(T * P.ld_d);
+    v.deq_x = take(T * 4);
+    v.u = take(T * P.E * 4);
+    v.q_u = take(T * P.ld_E);
+    v.deq_u = take(T * 4);
+    v.Bm = take(T * P.N * 4);
+    v.Cm = take(T * P.N * 4);
+    v.q_dt = take(T * P.ld_R);
+    v.deq_dt = take(T * 4);
+    v.y = take(T * P.E * 4);
+    v.q_y = take(T * P.ld_E);
+    v.deq_y = take(T * 4);
+  } else {
+    P.ss_parts = (P.E + rowss_bn(P.E) - 1) / rowss_bn(P.E);
+    v.r_x = take(T * 4);
+    v.u = take(T * P.E * 2);
+    P.ss_u = take(T * P.ss_parts * 4);
+    v.dt_low = take(T * P.ld_R * 2);
+    v.r_dt = take(T * 4);
+    v.Bm = take(T * P.N * 4);
+    v.Cm = take(T * P.N * 4);
+    v.delta_raw = take(T * P.E * 4);
+    v.y = take(T * P.E * 2);
+    v.r_y = take(T * 4);
+  }
+  P.total = a;
+  return P;
+}
+
+void fill_expand_jobs(const bitssm_layer* p, const LayerPlan& P, uint8_t* wbase, ExpandJobs& J) {
+  auto job = [&](int i, const bitssm_tw& w, int row0, size_t off, int ld) {
+    J.job[i].packed = w.packed;
+    J.job[i].scales = w.scales;
+    J.job[i].n_out = w.n_out;
+    J.job[i].k_in = w.k_in;
+    J.job[i].group = w.group;
+    J.job[i].row0 = row0;
+    J.job[i].dst = wbase + off;
+    J.job[i].ld = ld;
+  };
+  job(0, p->in_proj, 0, P.w_in, P.ld_d);
+  job(1, p->dt_down, 0, P.w_x, P.ld_E);
+  job(2, p->b_proj, P.R, P.w_x, P.ld_E);
+  job(3, p->c_proj, P.R + P.N, P.w_x, P.ld_E);
+  job(4, p->dt_up, 0, P.w_up, P.ld_R);
+  job(5, p->out_proj, 0, P.w_out, P.ld_E);
+  J.count = 6;
+}
+
+// Optional per-launch events: events[i] is recorded before the i-th kernel
+// of a forward and events[count] after the last one.
+struct Marks {
+  void* const* ev = nullptr;
+  int n = 0;
+  int i = 0;
+  cudaStream_t st = nullptr;
+  bool failed = false;
+  void mark() {
+    if (ev != nullptr && i < n) {
+      // Under stream capture the record must be an external event-record
+      // node of the graph (so graph replays can be timed); outside capture
+      // it is a plain record.
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      cudaError_t e = cudaStreamIsCapturing(st, &cs);
+      if (e == cudaSuccess) {
+        cudaEvent_t evt = reinterpret_cast<cudaEvent_t>(ev[i]);
+        e = cs == cudaStreamCaptureStatusActive
+                ? cudaEventRecordWithFlags(evt, st, cudaEventRecordExternal)
+                : cudaEventRecord(evt, st);
+      }
+      if (e != cudaSuccess) {
+        note_cuda_error(e);
+        failed = true;
+      }
+    }
+    ++i;
+  }
+};
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(base) + off);
+}
+
+int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, const void* x,
+               void* out, const void* residual, int B, int L, int dtype, void* ws,
+               cudaStream_t st, Marks& mk) {
+  const bitssm_ws_view& v = P.v;
+  const int T = P.T;
+  int rc;
+  // a1: RMSNorm + absmax int8 codes of x
+  mk.mark();
+  rc = launch_quant_rows(x, dtype, T, P.d, P.d, at<int8_t>(ws, v.q_x), P.ld_d, at<float>(ws, v.deq_x), st);
+  if (rc) return rc;
+  // a2 + a3: in_proj, u = acc * s_in * deq_x, codes of u from the int32 row
+  mk.mark();
+  {
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.E; G.K = P.d;
+    G.alpha = p->in_proj.scales;
+    G.row_scale = at<float>(ws, v.deq_x);
+    G.out = at<float>(ws, v.u); G.ld_out = P.E;
+    G.q_out = at<int8_t>(ws, v.q_u); G.ld_q = P.ld_E;
+    G.deq_out = at<float>(ws, v.deq_u);
+    rc = launch_gemm<false, EPI_QUANT_ROW>(at<int8_t>(ws, v.q_x), P.ld_d, wexp + P.w_in, P.ld_d, P.E, G, st);
+    if (rc) return rc;
+  }
+  // a4: x_proj (Delta-down | B | C), dt codes from the int32 row
+  mk.mark();
+  {
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.xrows; G.K = P.E;
+    G.row_scale = at<float>(ws, v.deq_u);
+    G.q_out = at<int8_t>(ws, v.q_dt); G.ld_q = P.ld_R;
+    G.deq_out = at<float>(ws, v.deq_dt);
+    G.R = P.R; G.Ns = P.N;
+    G.alpha_dt = p->dt_down.scales; G.alpha_B = p->b_proj.scales; G.alpha_C = p->c_proj.scales;
+    G.Bm = at<float>(ws, v.Bm); G.Cm = at<float>(ws, v.Cm);
+    rc = launch_gemm<false, EPI_XPROJ_A8>(at<int8_t>(ws, v.q_u), P.ld_E, wexp + P.w_x, P.ld_E, P.xrows, G, st);
+    if (rc) return rc;
+  }
+  // a5 + a6: Delta-up + softplus fused into the selective scan
+  mk.mark();
+  {
+    ScanParams S;
+    std::memset(&S, 0, sizeof(S));
+    S.u = at<float>(ws, v.u);
+    S.q_dt = at<int8_t>(ws, v.q_dt); S.ld_qdt = P.ld_R;
+    S.deq_dt = at<float>(ws, v.deq_dt);
+    S.W_up = reinterpret_cast<const int8_t*>(wexp + P.w_up); S.ld_w = P.ld_R;
+    S.s_up = p->dt_up.scales;
+    S.R = P.ld_R;
+    S.bias = p->dt_bias; S.A = p->A; S.D = p->D;
+    S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
+    S.y = at<float>(ws, v.y);
+    S.B = B; S.L = L; S.E = P.E;
+    rc = launch_scan<true, float, float, float>(S, st);
+    if (rc) return rc;
+  }
+  // a7: codes of y
+  mk.mark();
+  rc = launch_quant_rows(at<float>(ws, v.y), BITSSM_F32, T, P.E, P.E, at<int8_t>(ws, v.q_y), P.ld_E,
+                         at<float>(ws, v.deq_y), st);
+  if (rc) return rc;
+  // a8: out_proj (+ residual)
+  mk.mark();
+  {
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.d; G.K = P.E;
+    G.out_dtype = dtype;
+    G.alpha = p->out_proj.scales;
+    G.row_scale = at<float>(ws, v.deq_y);
+    G.out = out; G.ld_out = P.d;
+    G.residual = residual;
+    rc = launch_gemm<false, EPI_STORE>(at<int8_t>(ws, v.q_y), P.ld_E, wexp + P.w_out, P.ld_E, P.d, G, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  return BITSSM_OK;
+}
+
+int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, const void* x,
+                void* out, const void* residual, int B, int L, void* ws, cudaStream_t st,
+                Marks& mk) {
+  const bitssm_ws_view& v = P.v;
+  const int T = P.T;
+  int rc;
+  mk.mark();
+  rc = launch_row_rms(x, BITSSM_BF16, T, P.d, P.d, at<float>(ws, v.r_x), st);
+  if (rc) return rc;
+  mk.mark();
+  {  // in_proj: u = r_x * acc (bf16) + partial sum(u^2) per N tile
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.E; G.K = P.d;
+    G.row_scale = at<float>(ws, v.r_x);
+    G.out = at<__nv_bfloat16>(ws, v.u); G.ld_out = P.E;
+    G.ss_part = at<float>(ws, P.ss_u);
+    rc = launch_gemm<true, EPI_ROWSS>(x, P.d, wexp + P.w_in, P.ld_d, P.E, G, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  {  // x_proj: dt_low (bf16) + r_dt, B, C
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.xrows; G.K = P.E;
+    G.out = at<__nv_bfloat16>(ws, v.dt_low); G.ld_out = P.ld_R;
+    G.R = P.R; G.Ns = P.N;
+    G.Bm = at<float>(ws, v.Bm); G.Cm = at<float>(ws, v.Cm);
+    G.ss_in = at<float>(ws, P.ss_u); G.ss_nparts = P.ss_parts; G.ss_count = P.E;
+    G.r_out = at<float>(ws, v.r_dt);
+    rc = launch_gemm<true, EPI_XPROJ_A16>(at<__nv_bfloat16>(ws, v.u), P.E, wexp + P.w_x, P.ld_E,
+                                          P.xrows, G, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  {  // dt_proj: delta_raw = r_dt * acc (f32)
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.E; G.K = P.R;
+    G.out_dtype = BITSSM_F32;
+    G.row_scale = at<float>(ws, v.r_dt);
+    G.out = at<float>(ws, v.delta_raw); G.ld_out = P.E;
+    rc = launch_gemm<true, EPI_STORE>(at<__nv_bfloat16>(ws, v.dt_low), P.ld_R, wexp + P.w_up,
+                                      P.ld_R, P.E, G, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  {
+    ScanParams S;
+    std::memset(&S, 0, sizeof(S));
+    S.u = at<__nv_bfloat16>(ws, v.u);
+    S.delta_raw = at<float>(ws, v.delta_raw);
+    S.bias = p->dt_bias; S.A = p->A; S.D = p->D;
+    S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
+    S.y = at<__nv_bfloat16>(ws, v.y);
+    S.B = B; S.L = L; S.E = P.E;
+    rc = launch_scan<false, __nv_bfloat16, float, __nv_bfloat16>(S, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  rc = launch_row_rms(at<__nv_bfloat16>(ws, v.y), BITSSM_BF16, T, P.E, P.E, at<float>(ws, v.r_y), st);
+  if (rc) return rc;
+  mk.mark();
+  {
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = T; G.N = P.d; G.K = P.E;
+    G.out_dtype = BITSSM_BF16;
+    G.row_scale = at<float>(ws, v.r_y);
+    G.out = out; G.ld_out = P.d;
+    G.residual = residual;
+    rc = launch_gemm<true, EPI_STORE>(at<__nv_bfloat16>(ws, v.y), P.E, wexp + P.w_out, P.ld_E,
+                                      P.d, G, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  return BITSSM_OK;
+}
+
+int check_layer_args(const bitssm_layer* p, int B, int L, int dtype, int act_mode) {
+  if (act_mode != BITSSM_A8 && act_mode != BITSSM_A16) return BITSSM_ERR_INVALID_ARG;
+  if (dtype != BITSSM_F32 && dtype != BITSSM_BF16) return BITSSM_ERR_INVALID_ARG;
+  if (B < 0 || L < 0) return BITSSM_ERR_INVALID_ARG;
+  if (!layer_shape_ok(p, act_mode)) return BITSSM_ERR_INVALID_ARG;
+  if (act_mode == BITSSM_A16 && dtype != BITSSM_BF16) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if ((long)B * L > (1L << 30)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  return layer_supported(p, act_mode);
+}
+
+}  // namespace
+}  // namespace bitssm
+
+using namespace bitssm;
+
+extern "C" {
+
+int bitssm_version(void) { return BITSSM_ABI_VERSION; }
+
+const char* bitssm_last_error(void) { return g_last_error; }
+
+const char* bitssm_status_string(int status) {
+  switch (status) {
+    case BITSSM_OK: return "ok";
+    case BITSSM_ERR_INVALID_ARG: return "invalid argument";
+    case BITSSM_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BITSSM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case BITSSM_ERR_CUDA: return "CUDA error";
+    case BITSSM_ERR_TIMEOUT: return "bounded device wait ran out";
+    case BITSSM_ERR_DEVICE_FLAG: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+int bitssm_device_error(unsigned int* flags, int clear) {
+  if (flags == nullptr) return BITSSM_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BITSSM_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return BITSSM_ERR_CUDA;
+  *flags = v;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &z, sizeof(z)) != cudaSuccess) return BITSSM_ERR_CUDA;
+  }
+  return v ? BITSSM_ERR_TIMEOUT : BITSSM_OK;
+}
+
+// ---------------------------------------------------------------- packing
+int bitssm_pack_workspace_size(int n_out, int k_in, int group, size_t* bytes) {
+  if (bytes == nullptr || n_out <= 0 || k_in <= 0 || (group != 0 && group != 128))
+    return BITSSM_ERR_INVALID_ARG;
+  *bytes = group == 0 ? align_up(sizeof(double) * 1024) : 0;
+  return BITSSM_OK;
+}
+
+int bitssm_pack_ternary(const float* W, int n_out, int k_in, int group, uint8_t* packed,
+                        float* scales, void* ws, size_t ws_bytes, void* stream) {
+  if (W == nullptr || packed == nullptr || scales == nullptr || n_out <= 0 || k_in <= 0 ||
+      (group != 0 && group != 128))
+    return BITSSM_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (group == 0) {
+    size_t need = 0;
+    bitssm_pack_workspace_size(n_out, k_in, group, &need);
+    if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255))
+      return BITSSM_ERR_WORKSPACE;
+    const int nparts = 1024;
+    double* parts = reinterpret_cast<double*>(ws);
+    absmean_partial_kernel<<<nparts, 256, 0, st>>>(W, (long)n_out * k_in, parts);
+    const long nbytes = (long)n_out * ((k_in + 3) / 4);
+    long g = (nbytes + 255) / 256;
+    long cap = (long)num_sms() * 8;
+    pack_tensor_kernel<<<(int)(g < cap ? g : cap), 256, 0, st>>>(W, n_out, k_in, parts, nparts,
+                                                                packed, scales);
+  } else {
+    const long groups = (long)n_out * ((k_in + group - 1) / group);
+    long g = (groups + 7) / 8;
+    long cap = (long)num_sms() * 16;
+    pack_group_kernel<<<(int)(g < cap ? g : cap), 256, 0, st>>>(W, n_out, k_in, group, packed,
+                                                               scales);
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- BitLinear
+int bitlinear_workspace_size(const bitssm_tw* w, int M, int act_mode, size_t* bytes) {
+  if (bytes == nullptr || !tw_ok(w) || M < 0) return BITSSM_ERR_INVALID_ARG;
+  const int ld = round_up(w->k_in, 16);
+  if (act_mode == BITSSM_A8) {
+    *bytes = align_up((size_t)w->n_out * ld) + align_up((size_t)M * ld) + align_up((size_t)M * 4);
+  } else if (act_mode == BITSSM_A16) {
+    *bytes = align_up((size_t)w->n_out * ld * 2) + align_up((size_t)M * 4);
+  } else {
+    return BITSSM_ERR_INVALID_ARG;
+  }
+  return BITSSM_OK;
+}
+
+int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, void* y, int y_dtype,
+                      int act_mode, void* ws, size_t ws_bytes, void* stream) {
+  if (!tw_ok(w) || M < 0 || (M > 0 && (x == nullptr || y == nullptr)))
+    return BITSSM_ERR_INVALID_ARG;
+  if (x_dtype != BITSSM_F32 && x_dtype != BITSSM_BF16) return BITSSM_ERR_INVALID_ARG;
+  if (y_dtype != BITSSM_F32 && y_dtype != BITSSM_BF16 && y_dtype != BITSSM_I32)
+    return BITSSM_ERR_INVALID_ARG;
+  if (act_mode != BITSSM_A8 && act_mode != BITSSM_A16) return BITSSM_ERR_INVALID_ARG;
+  if (act_mode == BITSSM_A8 && w->group != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (act_mode == BITSSM_A16 && (x_dtype != BITSSM_BF16 || y_dtype == BITSSM_I32 || w->k_in % 8))
+    return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  size_t need = 0;
+  bitlinear_workspace_size(w, M, act_mode, &need);
+  if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return BITSSM_ERR_WORKSPACE;
+  if (M == 0) return BITSSM_OK;
+  cudaStream_t st = as_stream(stream);
+  const int ld = round_up(w->k_in, 16);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  ExpandJobs J;
+  std::memset(&J, 0, sizeof(J));
+  J.count = 1;
+  J.job[0].packed = w->packed;
+  J.job[0].scales = w->scales;
+  J.job[0].n_out = w->n_out;
+  J.job[0].k_in = w->k_in;
+  J.job[0].group = w->group;
+  J.job[0].row0 = 0;
+  J.job[0].dst = base;
+  J.job[0].ld = ld;
+  const bool a16 = act_mode == BITSSM_A16;
+  int rc = launch_expand(J, a16, st);
+  if (rc) return rc;
+  GemmParams G;
+  std::memset(&G, 0, sizeof(G));
+  G.M = M; G.N = w->n_out; G.K = w->k_in;
+  G.out = y; G.ld_out = w->n_out;
+  G.out_dtype = y_dtype;
+  if (!a16) {
+    int8_t* q = reinterpret_cast<int8_t*>(base + align_up((size_t)w->n_out * ld));
+    float* deq = reinterpret_cast<float*>(base + align_up((size_t)w->n_out * ld) + align_up((size_t)M * ld));
+    rc = launch_quant_rows(x, x_dtype, M, w->k_in, w->k_in, q, ld, deq, st);
+    if (rc) return rc;
+    G.alpha = w->scales;
+    G.row_scale = deq;
+    return launch_gemm<false, EPI_STORE>(q, ld, base, ld, w->n_out, G, st);
+  }
+  float* r = reinterpret_cast<float*>(base + align_up((size_t)w->n_out * ld * 2));
+  rc = launch_row_rms(x, BITSSM_BF16, M, w->k_in, w->k_in, r, st);
+  if (rc) return rc;
+  G.row_scale = r;
+  return launch_gemm<true, EPI_STORE>(x, w->k_in, base, ld, w->n_out, G, st);
+}
+
+// ---------------------------------------------------------------- scan
+int selective_scan_forward(const void* u, const void* delta_raw, const float* delta_bias,
+                           const float* A, const float* Bm, const float* Cm, const float* D,
+                           const float* h0, void* y, float* h_last, int B, int L, int E, int N,
+                           int dtype, void* stream) {
+  if (B < 0 || L < 0 || E <= 0 || N <= 0) return BITSSM_ERR_INVALID_ARG;
+  if (dtype != BITSSM_F32 && dtype != BITSSM_BF16) return BITSSM_ERR_INVALID_ARG;
+  if (N != kScanN) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || L == 0) {
+    if (h_last != nullptr && B > 0) {
+      cudaStream_t st = as_stream(stream);
+      const size_t bytes = (size_t)B * E * N * sizeof(float);
+      cudaError_t e = h0 != nullptr ? cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, st)
+                                    : cudaMemsetAsync(h_last, 0, bytes, st);
+      return e == cudaSuccess ? BITSSM_OK : BITSSM_ERR_CUDA;
+    }
+    return BITSSM_OK;
+  }
+  if (u == nullptr || delta_raw == nullptr || delta_bias == nullptr || A == nullptr ||
+      Bm == nullptr || Cm == nullptr || D == nullptr || y == nullptr)
+    return BITSSM_ERR_INVALID_ARG;
+  if (B > 65535) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  ScanParams S;
+  std::memset(&S, 0, sizeof(S));
+  S.u = u; S.delta_raw = delta_raw; S.bias = delta_bias; S.A = A; S.Bm = Bm; S.Cm = Cm; S.D = D;
+  S.h0 = h0; S.y = y; S.h_last = h_last; S.B = B; S.L = L; S.E = E;
+  cudaStream_t st = as_stream(stream);
+  if (dtype == BITSSM_F32) return launch_scan<false, float, float, float>(S, st);
+  return launch_scan<false, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(S, st);
+}
+
+// ---------------------------------------------------------------- layer
+int bitssm_prepared_size(const bitssm_layer* p, int act_mode, size_t* bytes) {
+  if (bytes == nullptr || (act_mode != BITSSM_A8 && act_mode != BITSSM_A16) ||
+      !layer_shape_ok(p, act_mode))
+    return BITSSM_ERR_INVALID_ARG;
+  *bytes = plan_layer(p, 1, 1, act_mode, false).w_bytes;
+  return BITSSM_OK;
+}
+
+int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_t dst_bytes,
+                           void* stream) {
+  size_t need = 0;
+  int rc = bitssm_prepared_size(p, act_mode, &need);
+  if (rc) return rc;
+  if (dst == nullptr || dst_bytes < need || (reinterpret_cast<uintptr_t>(dst) & 255))
+    return BITSSM_ERR_WORKSPACE;
+  LayerPlan P = plan_layer(p, 1, 1, act_mode, false);
+  ExpandJobs J;
+  std::memset(&J, 0, sizeof(J));
+  fill_expand_jobs(p, P, reinterpret_cast<uint8_t*>(dst), J);
+  return launch_expand(J, act_mode == BITSSM_A16, as_stream(stream));
+}
+
+int bitssm_workspace_size(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
+                          size_t* bytes) {
+  if (bytes == nullptr) return BITSSM_ERR_INVALID_ARG;
+  int rc = check_layer_args(p, B, L, dtype, act_mode);
+  if (rc) return rc;
+  *bytes = plan_layer(p, B, L, act_mode, p->prepared != nullptr).total;
+  return BITSSM_OK;
+}
+
+int bitssm_workspace_layout(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
+                            bitssm_ws_view* view) {
+  if (view == nullptr) return BITSSM_ERR_INVALID_ARG;
+  int rc = check_layer_args(p, B, L, dtype, act_mode);
+  if (rc) return rc;
+  *view = plan_layer(p, B, L, act_mode, p->prepared != nullptr).v;
+  return BITSSM_OK;
+}
+
+}  // extern "C"
+
+namespace bitssm {
+namespace {
+int forward_impl(const bitssm_layer* p, const void* x, void* out, const void* residual, int B,
+                 int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream,
+                 Marks& mk) {
+  int rc = check_layer_args(p, B, L, dtype, act_mode);
+  if (rc) return rc;
+  const long T = (long)B * L;
+  if (T > 0 && (x == nullptr || out == nullptr)) return BITSSM_ERR_INVALID_ARG;
+  const bool prepared = p->prepared != nullptr;
+  LayerPlan P = plan_layer(p, B, L, act_mode, prepared);
+  if (ws == nullptr || ws_bytes < P.total || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return BITSSM_ERR_WORKSPACE;
+  if (prepared && (reinterpret_cast<uintptr_t>(p->prepared) & 255)) return BITSSM_ERR_WORKSPACE;
+  if (T == 0) return BITSSM_OK;
+  cudaStream_t st = as_stream(stream);
+  mk.st = st;
+  const uint8_t* wexp;
+  if (prepared) {
+    wexp = reinterpret_cast<const uint8_t*>(p->prepared);
+  } else {
+    ExpandJobs J;
+    std::memset(&J, 0, sizeof(J));
+    fill_expand_jobs(p, P, reinterpret_cast<uint8_t*>(ws), J);
+    mk.mark();
+    rc = launch_expand(J, act_mode == BITSSM_A16, st);
+    if (rc) return rc;
+    wexp = reinterpret_cast<const uint8_t*>(ws);
+  }
+  rc = act_mode == BITSSM_A8 ? forward_a8(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk)
+                             : forward_a16(p, P, wexp, x, out, residual, B, L, ws, st, mk);
+  if (rc == BITSSM_OK && mk.failed) rc = BITSSM_ERR_CUDA;
+  return rc;
+}
+}  // namespace
+}  // namespace bitssm
+
+extern "C" {
+
+int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* residual, int B,
+                   int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream) {
+  Marks mk;
+  return forward_impl(p, x, out, residual, B, L, dtype, act_mode, ws, ws_bytes, stream, mk);
+}
+
+int bitssm_forward_launches(const bitssm_layer* p, int act_mode) {
+  if (p == nullptr || (act_mode != BITSSM_A8 && act_mode != BITSSM_A16)) return -1;
+  const int expand = p->prepared != nullptr ? 0 : 1;
+  return expand + (act_mode == BITSSM_A8 ? 6 : 7);
+}
+
+int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const void* residual,
+                         int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* const* events, int n_events, void* stream) {
+  const int nl = bitssm_forward_launches(p, act_mode);
+  if (nl < 0 || events == nullptr || n_events < nl + 1) return BITSSM_ERR_INVALID_ARG;
+  for (int i = 0; i <= nl; ++i)
+    if (events[i] == nullptr) return BITSSM_ERR_INVALID_ARG;
+  Marks mk;
+  mk.ev = events;
+  mk.n = n_events;
+  return forward_impl(p, x, out, residual, B, L, dtype, act_mode, ws, ws_bytes, stream, mk);
+}
+
+int bitssm_stack_forward(const bitssm_layer* layers, int n_layers, const void* x, void* out,
+                         int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (layers == nullptr || n_layers <= 0) return BITSSM_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_layer_args(&layers[l], B, L, dtype, act_mode);
+    if (rc) return rc;
+    if (layers[l].d_model != layers[0].d_model || layers[l].d_inner != layers[0].d_inner ||
+        layers[l].dt_rank != layers[0].dt_rank)
+      return BITSSM_ERR_INVALID_ARG;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    const void* in = l == 0 ? x : out;
+    int rc = bitssm_forward(&layers[l], in, out, in, B, L, dtype, act_mode, ws, ws_bytes, stream);
+    if (rc) return rc;
+  }
+  return BITSSM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,326 @@
+// Row-wise kernels: absmax int8 quantisation with the RMSNorm folded in,
+// the RMSNorm factor alone, absmean ternary packing, and the expansion of
+// packed ternary weights to tensor-core operand form.
+//
+// Quantiser (BitNet b1.58 BitLinear activations, TriSSM README opening
+// paragraph; an RMSNorm precedes each ternary projection, TriSSM README
+// caption "The BitSSM sequence mixer"):
+//   m = max|v|, sigma = fl32(127 / m), q = clamp(rint(fl32(v * sigma)), -128, 127)
+//   r = 1 / sqrt(mean(v^2) + eps),  deq = m * r / 127
+// Unit-gain RMSNorm scales a row by r > 0 and max|v r| = m r, so the codes of
+// the normalised row are the codes of v, and the dequantisation factor of
+// the normalised row's codes, expressed against v, is m r / 127.
+// The code decision uses IEEE round-to-nearest float32 division and
+// multiplication (__fdiv_rn, __fmul_rn) and round-half-to-even conversion,
+// never a contracted or approximate form.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace bitssm {
+
+constexpr float kEpsNorm = 1e-5f;
+constexpr float kEpsW = 1e-5f;
+
+template <typename T>
+__device__ __forceinline__ float load_as_float(const T* p);
+template <>
+__device__ __forceinline__ float load_as_float<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ int quant_code(float v, float sigma) {
+  int q = __float2int_rn(__fmul_rn(v, sigma));
+  return max(-128, min(127, q));
+}
+
+// One warp per row.  x [M, K] (row pitch ldx elements) -> q int8 [M, ldq]
+// (columns K..ldq-1 written as 0), deq [M].  The row is read twice (the
+// second time from L1/L2): once for max|v| and sum(v^2), once for the codes.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ x, int M, int K,
+                                                         long ldx, int8_t* __restrict__ q,
+                                                         long ldq, float* __restrict__ deq) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const T* xr = x + row * ldx;
+    float mx = 0.f, ss = 0.f;
+    for (int k = lane; k < K; k += 32) {
+      float v = load_as_float(xr + k);
+      mx = fmaxf(mx, fabsf(v));
+      ss = fmaf(v, v, ss);
+    }
+    mx = warp_max(mx);
+    ss = warp_sum(ss);
+    const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+    int8_t* qr = q + row * ldq;
+    // 4 codes per lane per step, written as one 32-bit word
+    for (int k0 = lane * 4; k0 < ldq; k0 += 128) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int k = k0 + j;
+        int c = 0;
+        if (k < K) c = quant_code(load_as_float(xr + k), sigma);
+        word |= (uint32_t)(c & 0xff) << (8 * j);
+      }
+      *reinterpret_cast<uint32_t*>(qr + k0) = word;
+    }
+    if (lane == 0) {
+      const float r = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
+      deq[row] = mx * r / 127.f;
+    }
+  }
+}
+
+// r[m] = 1 / sqrt(mean(x[m]^2) + eps), one warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256) row_rms_kernel(const T* __restrict__ x, int M, int K,
+                                                      long ldx, float* __restrict__ r) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const T* xr = x + row * ldx;
+    float ss = 0.f;
+    for (int k = lane; k < K; k += 32) {
+      float v = load_as_float(xr + k);
+      ss = fmaf(v, v, ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) r[row] = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Absmean ternary packing (BitNet b1.58 weights; grouped scales: Ternary
+// Mamba abstract).  s = mean|W| summed in float64 and rounded to float;
+// W_q = clip(rint(W / fl32(s + 1e-5)), -1, 1); code c = W_q + 1 at bits
+// 2*(k mod 4) of byte k/4, padding c = 1.
+// ---------------------------------------------------------------------------
+
+// Per-tensor scale, pass 1: `nparts` fixed partial sums of |W| in float64
+// (grid-stride over a fixed partition, so the summation order is fixed).
+__global__ void __launch_bounds__(256) absmean_partial_kernel(const float* __restrict__ W,
+                                                              long count,
+                                                              double* __restrict__ parts) {
+  __shared__ double red[8];
+  double acc = 0.0;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+       i += (long)gridDim.x * blockDim.x)
+    acc += fabs((double)W[i]);
+  acc = warp_sum_d(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    parts[blockIdx.x] = t;
+  }
+}
+
+__device__ __forceinline__ uint32_t ternary_code2(float w, float denom) {
+  int c = __float2int_rn(__fdiv_rn(w, denom));
+  c = max(-1, min(1, c));
+  return (uint32_t)(c + 1);
+}
+
+// Per-tensor scale, pass 2: every block sums the partials in the same order,
+// then packs one byte (4 codes) per thread.
+__global__ void __launch_bounds__(256) pack_tensor_kernel(const float* __restrict__ W, int n_out,
+                                                          int k_in, const double* __restrict__ parts,
+                                                          int nparts, uint8_t* __restrict__ packed,
+                                                          float* __restrict__ scales) {
+  __shared__ float s_sh;
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < nparts; ++i) t += parts[i];
+    s_sh = (float)(t / ((double)n_out * (double)k_in));
+    if (blockIdx.x == 0) scales[0] = s_sh;
+  }
+  __syncthreads();
+  const float denom = __fadd_rn(s_sh, kEpsW);
+  const int kb = (k_in + 3) / 4;
+  const long nbytes = (long)n_out * kb;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < nbytes;
+       i += (long)gridDim.x * blockDim.x) {
+    const long n = i / kb;
+    const int b = (int)(i - n * kb);
+    uint32_t byte = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = 4 * b + j;
+      uint32_t c = 1;
+      if (k < k_in) c = ternary_code2(W[n * k_in + k], denom);
+      byte |= c << (2 * j);
+    }
+    packed[i] = (uint8_t)byte;
+  }
+}
+
+// Grouped scales: one warp per (row, group); the group's float64 sum of |W|
+// is reduced across the warp, then the warp packs the group's codes.
+__global__ void __launch_bounds__(256) pack_group_kernel(const float* __restrict__ W, int n_out,
+                                                         int k_in, int group,
+                                                         uint8_t* __restrict__ packed,
+                                                         float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int ng = (k_in + group - 1) / group;
+  const int kb = (k_in + 3) / 4;
+  const long total = (long)n_out * ng;
+  const int warps = blockDim.x >> 5;
+  for (long gi = (long)blockIdx.x * warps + (threadIdx.x >> 5); gi < total;
+       gi += (long)gridDim.x * warps) {
+    const long n = gi / ng;
+    const int j = (int)(gi - n * ng);
+    const int k0 = j * group;
+    const int k1 = min(k_in, k0 + group);
+    double acc = 0.0;
+    for (int k = k0 + lane; k < k1; k += 32) acc += fabs((double)W[n * k_in + k]);
+    acc = warp_sum_d(acc);
+    const float s = (float)(acc / (double)(k1 - k0));
+    if (lane == 0) scales[gi] = s;
+    const float denom = __fadd_rn(s, kEpsW);
+    // group is a multiple of 4, so bytes never straddle groups
+    for (int b = k0 / 4 + lane; b < (k1 + 3) / 4; b += 32) {
+      uint32_t byte = 0;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int k = 4 * b + jj;
+        uint32_t c = 1;
+        if (k < k1) c = ternary_code2(W[n * k_in + k], denom);
+        byte |= c << (2 * jj);
+      }
+      packed[n * kb + b] = (uint8_t)byte;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Expansion of packed ternary weights to tensor-core operand rows.
+// ---------------------------------------------------------------------------
+
+// One expansion job: rows [row0, row0 + n_out) of a destination matrix with
+// row pitch ld elements; columns k_in..ld-1 are written as zero.
+struct ExpandJob {
+  const uint8_t* packed;
+  const float* scales;
+  int n_out, k_in, group;
+  int row0;
+  void* dst;
+  int ld;
+};
+struct ExpandJobs {
+  ExpandJob job[8];
+  int count;
+};
+
+// 16 codes (one 32-bit word of packed bytes) -> 16 int8 in a uint4.
+__device__ __forceinline__ uint4 expand16_i8(uint32_t p) {
+  // t_j holds, in byte b, the code of element 4b + j
+  const uint32_t t0 = p & 0x03030303u;
+  const uint32_t t1 = (p >> 2) & 0x03030303u;
+  const uint32_t t2 = (p >> 4) & 0x03030303u;
+  const uint32_t t3 = (p >> 6) & 0x03030303u;
+  const uint32_t a01 = __byte_perm(t0, t1, 0x5140);  // t0.b0 t1.b0 t0.b1 t1.b1
+  const uint32_t a23 = __byte_perm(t2, t3, 0x5140);
+  const uint32_t b01 = __byte_perm(t0, t1, 0x7362);  // t0.b2 t1.b2 t0.b3 t1.b3
+  const uint32_t b23 = __byte_perm(t2, t3, 0x7362);
+  uint4 o;
+  o.x = __byte_perm(a01, a23, 0x5410);  // elements 0..3
+  o.y = __byte_perm(a01, a23, 0x7632);  // elements 4..7
+  o.z = __byte_perm(b01, b23, 0x5410);  // elements 8..11
+  o.w = __byte_perm(b01, b23, 0x7632);  // elements 12..15
+  // c in {0,1,2} per byte -> c - 1 as int8: (c + 0x7f) ^ 0x80, no carries
+  o.x = (o.x + 0x7f7f7f7fu) ^ 0x80808080u;
+  o.y = (o.y + 0x7f7f7f7fu) ^ 0x80808080u;
+  o.z = (o.z + 0x7f7f7f7fu) ^ 0x80808080u;
+  o.w = (o.w + 0x7f7f7f7fu) ^ 0x80808080u;
+  return o;
+}
+
+// int8 expansion: each thread writes 16 consecutive elements of one row.
+__global__ void __launch_bounds__(256) expand_i8_kernel(ExpandJobs jobs) {
+  for (int ji = 0; ji < jobs.count; ++ji) {
+    const ExpandJob J = jobs.job[ji];
+    const int kb = (J.k_in + 3) / 4;
+    const int chunks = J.ld / 16;
+    const long total = (long)J.n_out * chunks;
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long)gridDim.x * blockDim.x) {
+      const long n = i / chunks;
+      const int ch = (int)(i - n * chunks);
+      const uint8_t* src = J.packed + n * kb;
+      uint32_t p = 0x55555555u;  // code 1 (w = 0) in every slot
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int byte = ch * 4 + b;
+        const uint32_t v = byte < kb ? src[byte] : 0x55u;
+        p = (p & ~(0xffu << (8 * b))) | (v << (8 * b));
+      }
+      uint4 o = expand16_i8(p);
+      // zero columns >= k_in (padding codes inside the last byte already are 0)
+      int8_t* dst = reinterpret_cast<int8_t*>(J.dst) + (long)(J.row0 + n) * J.ld + ch * 16;
+      *reinterpret_cast<uint4*>(dst) = o;
+    }
+  }
+}
+
+// bf16 expansion with the group scale folded in: element = w * bf16(s[n, k/group]).
+__global__ void __launch_bounds__(256) expand_bf16_kernel(ExpandJobs jobs) {
+  for (int ji = 0; ji < jobs.count; ++ji) {
+    const ExpandJob J = jobs.job[ji];
+    const int kb = (J.k_in + 3) / 4;
+    const int ng = J.group > 0 ? (J.k_in + J.group - 1) / J.group : 1;
+    const int chunks = J.ld / 8;
+    const long total = (long)J.n_out * chunks;
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long)gridDim.x * blockDim.x) {
+      const long n = i / chunks;
+      const int ch = (int)(i - n * chunks);
+      const uint8_t* src = J.packed + n * kb;
+      uint32_t out[4];
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        uint32_t pair = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int k = ch * 8 + e2 * 2 + h;
+          uint32_t bits = 0;
+          if (k < J.k_in) {
+            const int c = (src[k >> 2] >> (2 * (k & 3))) & 3;
+            const float s = J.group > 0 ? J.scales[n * ng + k / J.group] : J.scales[0];
+            const float w = (float)(c - 1) * __bfloat162float(__float2bfloat16_rn(s));
+            bits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(w));
+          }
+          pair |= bits << (16 * h);
+        }
+        out[e2] = pair;
+      }
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(J.dst) + (long)(J.row0 + n) * J.ld + ch * 8;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+  }
+}
+
+}  // namespace bitssm
