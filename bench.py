@@ -120,18 +120,16 @@ def scan_bytes_per_token(E, N, R_pad):
 
 
 def layer_bytes_per_token(wl):
-    """Algorithmic HBM bytes of the whole unfused A8 forward per token (each
-    kernel reads its inputs and writes its outputs once)."""
+    """Algorithmic HBM bytes per token of the fused A8 forward: the pre kernel
+    reads x and writes u (fp32), B, C, the dt codes and their factor; the scan
+    reads those and writes y (fp32); the post kernel reads y and writes out."""
     d, E, N = wl.d_model, wl.d_inner, wl.d_state
     Rp = (wl.dt_rank + 15) // 16 * 16
     io = 2 if wl.io_dtype == "bf16" else 4
-    quant_x = d * io + d + 4
-    in_proj = d + 4 + E * 4 + E + 4
-    x_proj = E + 4 + 2 * N * 4 + Rp + 4
+    pre = d * io + E * 4 + 2 * N * 4 + Rp + 4
     scan = scan_bytes_per_token(E, N, Rp)
-    quant_y = E * 4 + E + 4
-    out_proj = E + 4 + d * io
-    return quant_x + in_proj + x_proj + scan + quant_y + out_proj
+    post = E * 4 + d * io
+    return pre + scan + post
 
 
 # ---------------------------------------------------------------- our arm
@@ -294,11 +292,15 @@ def run_ours(args):
         return
 
     # ---------------- roofline of the dominant kernel
-    names_a8 = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_x_proj",
-                "selective_scan_fused_dt", "quant_rows_y", "gemm_out_proj"]
-    names = names_a8 if act == abi.A8 else ["expand_weights", "row_rms_x", "gemm_in_proj",
-                                            "gemm_x_proj", "gemm_dt_proj", "selective_scan",
-                                            "row_rms_y", "gemm_out_proj"]
+    if act == abi.A8 and nl in (3, 4):
+        names = ["expand_weights", "bitssm_pre(quant_x+in_proj+x_proj)",
+                 "selective_scan_fused_dt", "bitssm_post(quant_y+out_proj)"]
+    elif act == abi.A8:
+        names = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_x_proj",
+                 "selective_scan_fused_dt", "quant_rows_y", "gemm_out_proj"]
+    else:
+        names = ["expand_weights", "row_rms_x", "gemm_in_proj", "gemm_x_proj", "gemm_dt_proj",
+                 "selective_scan", "row_rms_y", "gemm_out_proj"]
     if nl == len(names) - 1:
         names = names[1:]
     avg_kernel_ms = [sum(kern_ms[li][i] for li in range(n_layers)) / (args.steps * n_layers)

@@ -86,7 +86,10 @@ typedef struct bitssm_tw {
  * `prepared` may point to a device buffer filled by bitssm_prepare_weights()
  * for this layer and act mode (the weights expanded to tensor-core operand
  * form), or be NULL: the forward then expands them into its workspace on
- * every call. */
+ * every call.  `flags`: 0, or BITSSM_KEEP_CODES to have the forward also
+ * store the int8 activation codes of x, u and y in its workspace (see
+ * bitssm_workspace_layout; for stage-by-stage checks). */
+#define BITSSM_KEEP_CODES 1
 typedef struct bitssm_layer {
   bitssm_tw in_proj, dt_down, b_proj, c_proj, dt_up, out_proj;
   const float* A;
@@ -97,6 +100,7 @@ typedef struct bitssm_layer {
   int d_state;
   int dt_rank;
   const void* prepared;
+  int flags;
 } bitssm_layer;
 
 /* Version of this ABI (BITSSM_ABI_VERSION). */
@@ -202,10 +206,12 @@ int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* 
                    int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels one bitssm_forward call launches for this layer and act
- * mode (A8: 6, A16: 7, plus 1 for the weight expansion when `prepared` is
- * NULL), or -1 for a bad argument.  A8 launch order: [expand] quantise x,
- * in_proj, x_proj, scan (with Delta-up fused), quantise y, out_proj.  A16:
- * [expand] RMS of x, in_proj, x_proj, dt_proj, scan, RMS of y, out_proj. */
+ * mode, or -1 for a bad argument.  A8 with d_model in {128, 256}, d_inner in
+ * {256, 512} and dt_rank + 2 d_state <= 64: 3 (pre = quantise x + in_proj +
+ * x_proj; scan with Delta-up fused; post = quantise y + out_proj); other A8
+ * shapes: 6 (quantise x, in_proj, x_proj, scan, quantise y, out_proj).
+ * A16: 7 (RMS of x, in_proj, x_proj, dt_proj, scan, RMS of y, out_proj).
+ * Plus 1 (first) for the weight expansion when `prepared` is NULL. */
 int bitssm_forward_launches(const bitssm_layer* p, int act_mode);
 
 /* bitssm_forward, additionally recording events[i] (cudaEvent_t handles
@@ -237,8 +243,9 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
 
 /* Inspection of the forward's intermediates inside a workspace (for
  * stage-by-stage checks).  Fills byte offsets into the workspace, or
- * (size_t)-1 for a buffer the act mode does not use, and the row pitch in
- * elements of each buffer.
+ * (size_t)-1 for a buffer the forward does not write (the A8 codes q_x,
+ * q_u and q_y are written only with BITSSM_KEEP_CODES when the layer runs
+ * as the fused kernels), and the row pitch in elements of each buffer.
  *   A8:  q_x int8 [T, ld_qx], deq_x float [T], u float [T, E],
  *        q_u int8 [T, ld_qu], deq_u float [T], Bm float [T, N],
  *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],

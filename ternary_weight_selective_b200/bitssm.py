@@ -28,6 +28,7 @@ ERR_DEVICE_FLAG = 6
 
 F32, BF16, I32 = 0, 1, 2
 A8, A16 = 0, 1
+KEEP_CODES = 1
 
 
 class BitssmError(RuntimeError):
@@ -62,7 +63,7 @@ class bitssm_layer(ctypes.Structure):
                 ("c_proj", bitssm_tw), ("dt_up", bitssm_tw), ("out_proj", bitssm_tw),
                 ("A", _vp), ("D", _vp), ("dt_bias", _vp),
                 ("d_model", _i), ("d_inner", _i), ("d_state", _i), ("dt_rank", _i),
-                ("prepared", _vp)]
+                ("prepared", _vp), ("flags", _i)]
 
 
 class bitssm_ws_view(ctypes.Structure):

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "bitssm.h"
+#include "kernel_fused.cuh"
 #include "kernel_gemm.cuh"
 #include "kernel_scan.cuh"
 #include "kernels_rows.cuh"
@@ -85,46 +86,95 @@ bool make_map(CUtensorMap* map, const void* ptr, bool bf16, long k, long rows, l
 }
 
 // ------------------------------------------------------------ GEMM launch
-template <bool kBF16, int BN, int EPI>
+template <int BN, int EPI>
 int launch_gemm_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
                    const GemmParams& P, cudaStream_t st) {
   constexpr int kStage = 128 * 128 + BN * 128;
   constexpr int kStages = (200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage);
-  using Cfg = GemmConfig<kBF16, BN, kStages, EPI>;
-  auto kern = ternary_gemm_kernel<kBF16, BN, kStages, EPI>;
+  // epilogue warps per TMEM quadrant: 128-column slices (x_proj keeps whole rows)
+  constexpr int kSplit = EPI == EPI_XPROJ_A8 ? 1 : (BN >= 256 ? BN / 128 : 1);
+  using Cfg = GemmConfig<BN, kStages, kSplit>;
+  auto kern = ternary_gemm_kernel<BN, kStages, EPI, kSplit>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
         cudaSuccess)
-      return BITSSM_ERR_CUDA;
+      return launch_status();
     attr_set = true;
   }
   CUtensorMap mA, mW;
-  if (!make_map(&mA, A, kBF16, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
-  if (!make_map(&mW, W, kBF16, P.K, w_rows, ldw, BN > 256 ? 256 : BN))
+  if (!make_map(&mA, A, false, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (!make_map(&mW, W, false, P.K, w_rows, ldw, BN > 256 ? 256 : BN))
     return BITSSM_ERR_UNSUPPORTED_SHAPE;
   dim3 grid((P.M + 127) / 128, (P.N + BN - 1) / BN);
-  kern<<<grid, 192, Cfg::kSmemBytes, st>>>(mA, mW, P);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mA, mW, P);
   return launch_status();
 }
 
-// N-tile choice: the smallest instantiated BN covering the columns the
+// int8 GEMM N tile: the smallest instantiated BN covering the columns the
 // epilogue needs in one tile (whole-row epilogues), else 256 with N tiling.
-template <bool kBF16, int EPI>
+template <int EPI>
 int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, const GemmParams& P,
                 cudaStream_t st) {
-  const int need = (EPI == EPI_STORE || EPI == EPI_ROWSS) ? (P.N < 256 ? P.N : 256) : P.N;
-  if (need <= 64) return launch_gemm_bn<kBF16, 64, EPI>(A, lda, W, ldw, w_rows, P, st);
-  if (need <= 128) return launch_gemm_bn<kBF16, 128, EPI>(A, lda, W, ldw, w_rows, P, st);
-  if (need <= 256) return launch_gemm_bn<kBF16, 256, EPI>(A, lda, W, ldw, w_rows, P, st);
+  const int need = EPI == EPI_STORE ? (P.N < 256 ? P.N : 256) : P.N;
+  if (need <= 64) return launch_gemm_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if (need <= 128) return launch_gemm_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if (need <= 256) return launch_gemm_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);
   if constexpr (EPI == EPI_QUANT_ROW) {
-    if (need <= 512) return launch_gemm_bn<kBF16, 512, EPI>(A, lda, W, ldw, w_rows, P, st);
+    if (need <= 512) return launch_gemm_bn<512, EPI>(A, lda, W, ldw, w_rows, P, st);
   }
   return BITSSM_ERR_UNSUPPORTED_SHAPE;
 }
 
-// N-tile width used by the A16 in_proj (its partial sums are per tile)
-inline int rowss_bn(int N) { return N <= 64 ? 64 : N <= 128 ? 128 : 256; }
+// W1.58A16 GEMM with exact fp32 group scales (transposed scales in P.s_t).
+template <int BN, int EPI>
+int launch_gemm_gs_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
+                      const GemmParams& P, cudaStream_t st) {
+  constexpr int kStage = 128 * 128 + BN * 128;
+  constexpr int kStages = (200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage);
+  using Cfg = GsConfig<BN, kStages>;
+  auto kern = ternary_gemm_gs_kernel<BN, kStages, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+        cudaSuccess)
+      return launch_status();
+    attr_set = true;
+  }
+  CUtensorMap mA, mW;
+  if (!make_map(&mA, A, true, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (!make_map(&mW, W, true, P.K, w_rows, ldw, BN)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  dim3 grid((P.M + 127) / 128, (P.N + BN - 1) / BN);
+  kern<<<grid, 320, Cfg::kSmemBytes, st>>>(mA, mW, P);
+  return launch_status();
+}
+
+// N tile of the group-scaled GEMM: whole-row epilogues need every column in
+// one tile (and the dt columns within the first half).
+inline int gs_bn(int N, bool whole_row) {
+  const int need = whole_row ? N : (N < 256 ? N : 256);
+  return need <= 64 ? 64 : need <= 128 ? 128 : 256;
+}
+
+template <int EPI>
+int launch_gemm_gs(const void* A, long lda, const void* W, long ldw, long w_rows,
+                   const GemmParams& P, cudaStream_t st) {
+  const bool whole = EPI == EPI_XPROJ_A16;
+  if (whole && P.N > 256) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  const int bn = gs_bn(P.N, whole);
+  if (whole && P.R > bn / 2) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (bn == 64) return launch_gemm_gs_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if (bn == 128) return launch_gemm_gs_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
+  return launch_gemm_gs_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);
+}
+
+// Partial sums of u^2 per A16 in_proj row: two per N tile (one per epilogue
+// column half).
+inline int rowss_parts(int E) { return 2 * ((E + gs_bn(E, false) - 1) / gs_bn(E, false)); }
+
+// Transposed fp32 group scales of an expanded bf16 matrix: [G][ld_s]
+inline int scale_groups(int k_in) { return (k_in + 127) / 128; }
+inline long scale_ld(int rows) { return (long)round_up(rows, 256); }
 
 // ------------------------------------------------------------ row kernels
 inline int rows_grid(long M) {
@@ -133,9 +183,27 @@ inline int rows_grid(long M) {
   return (int)(g < cap ? (g < 1 ? 1 : g) : cap);
 }
 
+template <typename T>
+bool launch_quant_rows_vec(const void* x, int M, int K, long ldx, int8_t* q, long ldq, float* deq,
+                           cudaStream_t st) {
+  constexpr int EPV = 16 / (int)sizeof(T);
+  if (K % EPV || ldx % EPV || (reinterpret_cast<uintptr_t>(x) & 15) || (ldq % 8)) return false;
+  const int vpl = (K + 32 * EPV - 1) / (32 * EPV);
+  const T* xp = reinterpret_cast<const T*>(x);
+  if (vpl == 1) quant_rows_vec_kernel<T, 1><<<rows_grid(M), 256, 0, st>>>(xp, M, K, ldx, q, ldq, deq);
+  else if (vpl == 2) quant_rows_vec_kernel<T, 2><<<rows_grid(M), 256, 0, st>>>(xp, M, K, ldx, q, ldq, deq);
+  else if (vpl <= 4) quant_rows_vec_kernel<T, 4><<<rows_grid(M), 256, 0, st>>>(xp, M, K, ldx, q, ldq, deq);
+  else return false;
+  return true;
+}
+
 int launch_quant_rows(const void* x, int dtype, int M, int K, long ldx, int8_t* q, long ldq,
                       float* deq, cudaStream_t st) {
   if (M == 0) return BITSSM_OK;
+  const bool vec = dtype == BITSSM_F32
+                       ? launch_quant_rows_vec<float>(x, M, K, ldx, q, ldq, deq, st)
+                       : launch_quant_rows_vec<__nv_bfloat16>(x, M, K, ldx, q, ldq, deq, st);
+  if (vec) return launch_status();
   if (dtype == BITSSM_F32)
     quant_rows_kernel<float><<<rows_grid(M), 256, 0, st>>>(reinterpret_cast<const float*>(x), M, K,
                                                            ldx, q, ldq, deq);
@@ -158,40 +226,62 @@ int launch_row_rms(const void* x, int dtype, int M, int K, long ldx, float* r, c
 
 int launch_expand(const ExpandJobs& jobs, bool bf16, cudaStream_t st) {
   long total = 0;
-  for (int i = 0; i < jobs.count; ++i)
+  int first[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int i = 0; i < jobs.count; ++i) {
+    first[i] = (int)total;
     total += (long)jobs.job[i].n_out * (jobs.job[i].ld / (bf16 ? 8 : 16));
+  }
+  if (jobs.count < 8) first[jobs.count] = (int)total;
   long g = (total + 255) / 256;
   long cap = (long)num_sms() * 8;
   int grid = (int)(g < 1 ? 1 : (g < cap ? g : cap));
   if (bf16) expand_bf16_kernel<<<grid, 256, 0, st>>>(jobs);
-  else expand_i8_kernel<<<grid, 256, 0, st>>>(jobs);
+  else
+    expand_i8_kernel<<<grid, 256, 0, st>>>(jobs, make_int4(first[0], first[1], first[2], first[3]),
+                                           make_int4(first[4], first[5], first[6], first[7]));
   return launch_status();
 }
 
 // ------------------------------------------------------------ scan launch
-template <int NPT, bool FUSED, typename Tu, typename Td, typename Ty>
+template <int NPT, bool FUSED, int RV, typename Tu, typename Td, typename Ty>
 int launch_scan_t(const ScanParams& P, cudaStream_t st) {
-  constexpr int CE = 128 * NPT / kScanN;
-  const int Rm = FUSED ? P.R : 0;
-  const int smem = scan_smem_bytes(CE, Rm);
-  auto kern = selective_scan_kernel<NPT, FUSED, Tu, Td, Ty>;
-  if (smem > 48 * 1024) {
+  constexpr int TPC = kScanN / NPT;
+  constexpr int CE = 128 / TPC;
+  constexpr int smem = 2 * ScanStage<CE, FUSED, Tu, Td>::kBytes;
+  auto kern = selective_scan_kernel<NPT, FUSED, RV, Tu, Td, Ty>;
+  static bool attr_set = false;
+  if (!attr_set && smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return BITSSM_ERR_CUDA;
+      return launch_status();
+    attr_set = true;
   }
-  dim3 grid((P.E + CE - 1) / CE, P.B);
+  dim3 grid((unsigned)((P.E + CE - 1) / CE), (unsigned)P.B);
   kern<<<grid, 128, smem, st>>>(P);
   return launch_status();
 }
 
-// states per thread: enough threads to fill the machine when B*E is small
+// States per thread: 16 (one thread per channel, no exchange) when there are
+// enough channels to give every SM sub-partition ~1.5 warps, else 8 or 4.
+template <bool FUSED, int RV, typename Tu, typename Td, typename Ty>
+int launch_scan_rv(const ScanParams& P, cudaStream_t st) {
+  const long channels = (long)P.B * P.E;
+  const long want = (long)num_sms() * 4 * 48;
+  if (channels >= want) return launch_scan_t<16, FUSED, RV, Tu, Td, Ty>(P, st);
+  if (channels * 2 >= want) return launch_scan_t<8, FUSED, RV, Tu, Td, Ty>(P, st);
+  return launch_scan_t<4, FUSED, RV, Tu, Td, Ty>(P, st);
+}
+
 template <bool FUSED, typename Tu, typename Td, typename Ty>
 int launch_scan(const ScanParams& P, cudaStream_t st) {
-  const long channels = (long)P.B * P.E;
-  const long want = (long)num_sms() * 4 * 32 * 6;  // ~6 warps per SM sub-partition
-  if (channels * 16 / 16 >= want) return launch_scan_t<16, FUSED, Tu, Td, Ty>(P, st);
-  if (channels * 16 / 4 >= want) return launch_scan_t<4, FUSED, Tu, Td, Ty>(P, st);
-  return launch_scan_t<1, FUSED, Tu, Td, Ty>(P, st);
+  if constexpr (FUSED) {
+    switch (P.R / 16) {  // Delta-up width (dt_rank padded to 16)
+      case 1: return launch_scan_rv<true, 1, Tu, Td, Ty>(P, st);
+      case 2: return launch_scan_rv<true, 2, Tu, Td, Ty>(P, st);
+      case 3: case 4: return launch_scan_rv<true, 4, Tu, Td, Ty>(P, st);
+      default: return launch_scan_rv<true, 8, Tu, Td, Ty>(P, st);
+    }
+  }
+  return launch_scan_rv<false, 1, Tu, Td, Ty>(P, st);
 }
 
 // ------------------------------------------------------------ validation
@@ -208,6 +298,8 @@ struct LayerPlan {
   bool a16;
   // expanded weights (offsets relative to the expanded block)
   size_t w_in, w_x, w_up, w_out, w_bytes;
+  // A16: transposed fp32 group scales inside the expanded block
+  size_t s_in, s_x, s_up, s_out;
   // workspace offsets (absolute; expanded block at 0 when not prepared)
   size_t base;
   bitssm_ws_view v;
@@ -269,6 +361,12 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   P.w_x = o; o = align_up(o + (size_t)P.xrows * P.ld_E * es);
   P.w_up = o; o = align_up(o + (size_t)P.E * P.ld_R * es);
   P.w_out = o; o = align_up(o + (size_t)P.d * P.ld_E * es);
+  if (P.a16) {
+    P.s_in = o; o = align_up(o + (size_t)scale_groups(P.d) * scale_ld(P.E) * 4);
+    P.s_x = o; o = align_up(o + (size_t)scale_groups(P.E) * scale_ld(P.xrows) * 4);
+    P.s_up = o; o = align_up(o + (size_t)scale_groups(P.R) * scale_ld(P.E) * 4);
+    P.s_out = o; o = align_up(o + (size_t)scale_groups(P.E) * scale_ld(P.d) * 4);
+  }
   P.w_bytes = o;
   size_t a = prepared ? 0 : P.w_bytes;
   const size_t T = (size_t)P.T;
@@ -299,7 +397,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
     v.q_y = take(T * P.ld_E);
     v.deq_y = take(T * 4);
   } else {
-    P.ss_parts = (P.E + rowss_bn(P.E) - 1) / rowss_bn(P.E);
+    P.ss_parts = rowss_parts(P.E);
     v.r_x = take(T * 4);
     v.u = take(T * P.E * 2);
     P.ss_u = take(T * P.ss_parts * 4);
@@ -316,7 +414,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
 }
 
 void fill_expand_jobs(const bitssm_layer* p, const LayerPlan& P, uint8_t* wbase, ExpandJobs& J) {
-  auto job = [&](int i, const bitssm_tw& w, int row0, size_t off, int ld) {
+  auto job = [&](int i, const bitssm_tw& w, int row0, size_t off, int ld, size_t soff, long ld_s) {
     J.job[i].packed = w.packed;
     J.job[i].scales = w.scales;
     J.job[i].n_out = w.n_out;
@@ -325,14 +423,29 @@ void fill_expand_jobs(const bitssm_layer* p, const LayerPlan& P, uint8_t* wbase,
     J.job[i].row0 = row0;
     J.job[i].dst = wbase + off;
     J.job[i].ld = ld;
+    J.job[i].s_t = P.a16 ? reinterpret_cast<float*>(wbase + soff) : nullptr;
+    J.job[i].ld_s = ld_s;
   };
-  job(0, p->in_proj, 0, P.w_in, P.ld_d);
-  job(1, p->dt_down, 0, P.w_x, P.ld_E);
-  job(2, p->b_proj, P.R, P.w_x, P.ld_E);
-  job(3, p->c_proj, P.R + P.N, P.w_x, P.ld_E);
-  job(4, p->dt_up, 0, P.w_up, P.ld_R);
-  job(5, p->out_proj, 0, P.w_out, P.ld_E);
+  job(0, p->in_proj, 0, P.w_in, P.ld_d, P.s_in, scale_ld(P.E));
+  job(1, p->dt_down, 0, P.w_x, P.ld_E, P.s_x, scale_ld(P.xrows));
+  job(2, p->b_proj, P.R, P.w_x, P.ld_E, P.s_x, scale_ld(P.xrows));
+  job(3, p->c_proj, P.R + P.N, P.w_x, P.ld_E, P.s_x, scale_ld(P.xrows));
+  job(4, p->dt_up, 0, P.w_up, P.ld_R, P.s_up, scale_ld(P.E));
+  job(5, p->out_proj, 0, P.w_out, P.ld_E, P.s_out, scale_ld(P.d));
   J.count = 6;
+}
+
+// Expansion of a layer's weights into `wbase` (A16: the padding rows of the
+// transposed scales are zeroed first).
+int expand_layer(const bitssm_layer* p, const LayerPlan& P, uint8_t* wbase, cudaStream_t st) {
+  if (P.a16) {
+    if (cudaMemsetAsync(wbase + P.s_in, 0, P.w_bytes - P.s_in, st) != cudaSuccess)
+      return launch_status();
+  }
+  ExpandJobs J;
+  std::memset(&J, 0, sizeof(J));
+  fill_expand_jobs(p, P, wbase, J);
+  return launch_expand(J, P.a16, st);
 }
 
 // Optional per-launch events: events[i] is recorded before the i-th kernel
@@ -370,6 +483,126 @@ T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(base) + off);
 }
 
+// Whether the A8 layer runs as the fused pre kernel + scan + post kernel:
+// d_model of 128 or 256, d_inner of 256 or 512, dt_rank + 2 d_state <= 64.
+bool a8_fused(const LayerPlan& P) {
+  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64;
+}
+
+template <typename Tx, int BN1, int K1P>
+int launch_pre_t(const PreParams& Q, const void* w_in, long ld_in, const void* w_x, long ld_x,
+                 int xrows, cudaStream_t st) {
+  using Cfg = PreCfg<BN1, K1P, 64>;
+  auto kern = bitssm_pre_kernel<Tx, BN1, K1P, 64>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+      return launch_status();
+    attr_set = true;
+  }
+  CUtensorMap mWin, mWx;
+  if (!make_map(&mWin, w_in, false, Q.d, Q.E, ld_in, BN1 > 256 ? 256 : BN1)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (!make_map(&mWx, w_x, false, Q.E, xrows, ld_x, 64)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  kern<<<(Q.M + 127) / 128, kFusedThreads, Cfg::kSmemBytes, st>>>(mWin, mWx, Q);
+  return launch_status();
+}
+
+template <typename Tx>
+int launch_pre(const PreParams& Q, const void* w_in, long ld_in, const void* w_x, long ld_x,
+               int xrows, cudaStream_t st) {
+  if (Q.E == 512) {
+    if (Q.d == 256) return launch_pre_t<Tx, 512, 2>(Q, w_in, ld_in, w_x, ld_x, xrows, st);
+    return launch_pre_t<Tx, 512, 1>(Q, w_in, ld_in, w_x, ld_x, xrows, st);
+  }
+  if (Q.d == 256) return launch_pre_t<Tx, 256, 2>(Q, w_in, ld_in, w_x, ld_x, xrows, st);
+  return launch_pre_t<Tx, 256, 1>(Q, w_in, ld_in, w_x, ld_x, xrows, st);
+}
+
+template <int OUT_BF16, int BN, int KP>
+int launch_post_t(const PostParams& Q, const void* w, long ldw, cudaStream_t st) {
+  using Cfg = PostCfg<BN, KP>;
+  auto kern = bitssm_post_kernel<OUT_BF16, BN, KP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
+      return launch_status();
+    attr_set = true;
+  }
+  CUtensorMap mW;
+  if (!make_map(&mW, w, false, Q.E, Q.d, ldw, BN)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  kern<<<(Q.M + 127) / 128, kFusedThreads, Cfg::kSmemBytes, st>>>(mW, Q);
+  return launch_status();
+}
+
+template <int OUT_BF16>
+int launch_post(const PostParams& Q, const void* w, long ldw, cudaStream_t st) {
+  if (Q.E == 512) {
+    if (Q.d == 256) return launch_post_t<OUT_BF16, 256, 4>(Q, w, ldw, st);
+    return launch_post_t<OUT_BF16, 128, 4>(Q, w, ldw, st);
+  }
+  if (Q.d == 256) return launch_post_t<OUT_BF16, 256, 2>(Q, w, ldw, st);
+  return launch_post_t<OUT_BF16, 128, 2>(Q, w, ldw, st);
+}
+
+int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp,
+                     const void* x, void* out, const void* residual, int B, int L, int dtype,
+                     void* ws, cudaStream_t st, Marks& mk) {
+  const bitssm_ws_view& v = P.v;
+  const bool keep = (p->flags & BITSSM_KEEP_CODES) != 0;
+  int rc;
+  mk.mark();
+  {
+    PreParams Q;
+    std::memset(&Q, 0, sizeof(Q));
+    Q.x = x; Q.M = P.T; Q.d = P.d; Q.E = P.E; Q.xrows = P.xrows; Q.R = P.R; Q.Ns = P.N;
+    Q.s_in = p->in_proj.scales; Q.s_dt = p->dt_down.scales; Q.s_B = p->b_proj.scales;
+    Q.s_C = p->c_proj.scales;
+    Q.u = at<float>(ws, v.u); Q.deq_x = at<float>(ws, v.deq_x); Q.deq_u = at<float>(ws, v.deq_u);
+    Q.q_dt = at<int8_t>(ws, v.q_dt); Q.ld_qdt = P.ld_R; Q.deq_dt = at<float>(ws, v.deq_dt);
+    Q.Bm = at<float>(ws, v.Bm); Q.Cm = at<float>(ws, v.Cm);
+    if (keep) {
+      Q.q_x = at<int8_t>(ws, v.q_x); Q.ld_qx = P.ld_d;
+      Q.q_u = at<int8_t>(ws, v.q_u); Q.ld_qu = P.ld_E;
+    }
+    rc = dtype == BITSSM_F32
+             ? launch_pre<float>(Q, wexp + P.w_in, P.ld_d, wexp + P.w_x, P.ld_E, P.xrows, st)
+             : launch_pre<__nv_bfloat16>(Q, wexp + P.w_in, P.ld_d, wexp + P.w_x, P.ld_E, P.xrows, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  {
+    ScanParams S;
+    std::memset(&S, 0, sizeof(S));
+    S.u = at<float>(ws, v.u);
+    S.q_dt = at<int8_t>(ws, v.q_dt); S.ld_qdt = P.ld_R;
+    S.deq_dt = at<float>(ws, v.deq_dt);
+    S.W_up = reinterpret_cast<const int8_t*>(wexp + P.w_up); S.ld_w = P.ld_R;
+    S.s_up = p->dt_up.scales;
+    S.R = P.ld_R;
+    S.bias = p->dt_bias; S.A = p->A; S.D = p->D;
+    S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
+    S.y = at<float>(ws, v.y);
+    S.B = B; S.L = L; S.E = P.E;
+    rc = launch_scan<true, float, float, float>(S, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  {
+    PostParams Q;
+    std::memset(&Q, 0, sizeof(Q));
+    Q.y = at<float>(ws, v.y); Q.M = P.T; Q.E = P.E; Q.d = P.d;
+    Q.s_out = p->out_proj.scales;
+    Q.out = out; Q.residual = residual;
+    Q.deq_y = at<float>(ws, v.deq_y);
+    if (keep) { Q.q_y = at<int8_t>(ws, v.q_y); Q.ld_qy = P.ld_E; }
+    rc = dtype == BITSSM_F32 ? launch_post<0>(Q, wexp + P.w_out, P.ld_E, st)
+                             : launch_post<1>(Q, wexp + P.w_out, P.ld_E, st);
+    if (rc) return rc;
+  }
+  mk.mark();
+  return BITSSM_OK;
+}
+
 int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, const void* x,
                void* out, const void* residual, int B, int L, int dtype, void* ws,
                cudaStream_t st, Marks& mk) {
@@ -391,7 +624,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     G.out = at<float>(ws, v.u); G.ld_out = P.E;
     G.q_out = at<int8_t>(ws, v.q_u); G.ld_q = P.ld_E;
     G.deq_out = at<float>(ws, v.deq_u);
-    rc = launch_gemm<false, EPI_QUANT_ROW>(at<int8_t>(ws, v.q_x), P.ld_d, wexp + P.w_in, P.ld_d, P.E, G, st);
+    rc = launch_gemm<EPI_QUANT_ROW>(at<int8_t>(ws, v.q_x), P.ld_d, wexp + P.w_in, P.ld_d, P.E, G, st);
     if (rc) return rc;
   }
   // a4: x_proj (Delta-down | B | C), dt codes from the int32 row
@@ -406,7 +639,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     G.R = P.R; G.Ns = P.N;
     G.alpha_dt = p->dt_down.scales; G.alpha_B = p->b_proj.scales; G.alpha_C = p->c_proj.scales;
     G.Bm = at<float>(ws, v.Bm); G.Cm = at<float>(ws, v.Cm);
-    rc = launch_gemm<false, EPI_XPROJ_A8>(at<int8_t>(ws, v.q_u), P.ld_E, wexp + P.w_x, P.ld_E, P.xrows, G, st);
+    rc = launch_gemm<EPI_XPROJ_A8>(at<int8_t>(ws, v.q_u), P.ld_E, wexp + P.w_x, P.ld_E, P.xrows, G, st);
     if (rc) return rc;
   }
   // a5 + a6: Delta-up + softplus fused into the selective scan
@@ -443,7 +676,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     G.row_scale = at<float>(ws, v.deq_y);
     G.out = out; G.ld_out = P.d;
     G.residual = residual;
-    rc = launch_gemm<false, EPI_STORE>(at<int8_t>(ws, v.q_y), P.ld_E, wexp + P.w_out, P.ld_E, P.d, G, st);
+    rc = launch_gemm<EPI_STORE>(at<int8_t>(ws, v.q_y), P.ld_E, wexp + P.w_out, P.ld_E, P.d, G, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -467,7 +700,8 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     G.row_scale = at<float>(ws, v.r_x);
     G.out = at<__nv_bfloat16>(ws, v.u); G.ld_out = P.E;
     G.ss_part = at<float>(ws, P.ss_u);
-    rc = launch_gemm<true, EPI_ROWSS>(x, P.d, wexp + P.w_in, P.ld_d, P.E, G, st);
+    G.s_t = reinterpret_cast<const float*>(wexp + P.s_in); G.ld_s = scale_ld(P.E);
+    rc = launch_gemm_gs<EPI_ROWSS>(x, P.d, wexp + P.w_in, P.ld_d, P.E, G, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -480,8 +714,9 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     G.Bm = at<float>(ws, v.Bm); G.Cm = at<float>(ws, v.Cm);
     G.ss_in = at<float>(ws, P.ss_u); G.ss_nparts = P.ss_parts; G.ss_count = P.E;
     G.r_out = at<float>(ws, v.r_dt);
-    rc = launch_gemm<true, EPI_XPROJ_A16>(at<__nv_bfloat16>(ws, v.u), P.E, wexp + P.w_x, P.ld_E,
-                                          P.xrows, G, st);
+    G.s_t = reinterpret_cast<const float*>(wexp + P.s_x); G.ld_s = scale_ld(P.xrows);
+    rc = launch_gemm_gs<EPI_XPROJ_A16>(at<__nv_bfloat16>(ws, v.u), P.E, wexp + P.w_x, P.ld_E,
+                                       P.xrows, G, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -492,8 +727,9 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     G.out_dtype = BITSSM_F32;
     G.row_scale = at<float>(ws, v.r_dt);
     G.out = at<float>(ws, v.delta_raw); G.ld_out = P.E;
-    rc = launch_gemm<true, EPI_STORE>(at<__nv_bfloat16>(ws, v.dt_low), P.ld_R, wexp + P.w_up,
-                                      P.ld_R, P.E, G, st);
+    G.s_t = reinterpret_cast<const float*>(wexp + P.s_up); G.ld_s = scale_ld(P.E);
+    rc = launch_gemm_gs<EPI_STORE>(at<__nv_bfloat16>(ws, v.dt_low), P.ld_R, wexp + P.w_up, P.ld_R,
+                                   P.E, G, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -521,8 +757,9 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     G.row_scale = at<float>(ws, v.r_y);
     G.out = out; G.ld_out = P.d;
     G.residual = residual;
-    rc = launch_gemm<true, EPI_STORE>(at<__nv_bfloat16>(ws, v.y), P.E, wexp + P.w_out, P.ld_E,
-                                      P.d, G, st);
+    G.s_t = reinterpret_cast<const float*>(wexp + P.s_out); G.ld_s = scale_ld(P.d);
+    rc = launch_gemm_gs<EPI_STORE>(at<__nv_bfloat16>(ws, v.y), P.E, wexp + P.w_out, P.ld_E, P.d,
+                                   G, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -620,7 +857,9 @@ int bitlinear_workspace_size(const bitssm_tw* w, int M, int act_mode, size_t* by
   if (act_mode == BITSSM_A8) {
     *bytes = align_up((size_t)w->n_out * ld) + align_up((size_t)M * ld) + align_up((size_t)M * 4);
   } else if (act_mode == BITSSM_A16) {
-    *bytes = align_up((size_t)w->n_out * ld * 2) + align_up((size_t)M * 4);
+    *bytes = align_up((size_t)w->n_out * ld * 2) +
+             align_up((size_t)scale_groups(w->k_in) * scale_ld(w->n_out) * 4) +
+             align_up((size_t)M * 4);
   } else {
     return BITSSM_ERR_INVALID_ARG;
   }
@@ -646,6 +885,9 @@ int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, voi
   cudaStream_t st = as_stream(stream);
   const int ld = round_up(w->k_in, 16);
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  const bool a16 = act_mode == BITSSM_A16;
+  const size_t w_bytes = align_up((size_t)w->n_out * ld * (a16 ? 2 : 1));
+  const size_t s_bytes = a16 ? align_up((size_t)scale_groups(w->k_in) * scale_ld(w->n_out) * 4) : 0;
   ExpandJobs J;
   std::memset(&J, 0, sizeof(J));
   J.count = 1;
@@ -657,7 +899,11 @@ int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, voi
   J.job[0].row0 = 0;
   J.job[0].dst = base;
   J.job[0].ld = ld;
-  const bool a16 = act_mode == BITSSM_A16;
+  if (a16) {
+    J.job[0].s_t = reinterpret_cast<float*>(base + w_bytes);
+    J.job[0].ld_s = scale_ld(w->n_out);
+    if (cudaMemsetAsync(base + w_bytes, 0, s_bytes, st) != cudaSuccess) return launch_status();
+  }
   int rc = launch_expand(J, a16, st);
   if (rc) return rc;
   GemmParams G;
@@ -666,19 +912,21 @@ int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, voi
   G.out = y; G.ld_out = w->n_out;
   G.out_dtype = y_dtype;
   if (!a16) {
-    int8_t* q = reinterpret_cast<int8_t*>(base + align_up((size_t)w->n_out * ld));
-    float* deq = reinterpret_cast<float*>(base + align_up((size_t)w->n_out * ld) + align_up((size_t)M * ld));
+    int8_t* q = reinterpret_cast<int8_t*>(base + w_bytes);
+    float* deq = reinterpret_cast<float*>(base + w_bytes + align_up((size_t)M * ld));
     rc = launch_quant_rows(x, x_dtype, M, w->k_in, w->k_in, q, ld, deq, st);
     if (rc) return rc;
     G.alpha = w->scales;
     G.row_scale = deq;
-    return launch_gemm<false, EPI_STORE>(q, ld, base, ld, w->n_out, G, st);
+    return launch_gemm<EPI_STORE>(q, ld, base, ld, w->n_out, G, st);
   }
-  float* r = reinterpret_cast<float*>(base + align_up((size_t)w->n_out * ld * 2));
+  float* r = reinterpret_cast<float*>(base + w_bytes + s_bytes);
   rc = launch_row_rms(x, BITSSM_BF16, M, w->k_in, w->k_in, r, st);
   if (rc) return rc;
   G.row_scale = r;
-  return launch_gemm<true, EPI_STORE>(x, w->k_in, base, ld, w->n_out, G, st);
+  G.s_t = reinterpret_cast<const float*>(base + w_bytes);
+  G.ld_s = scale_ld(w->n_out);
+  return launch_gemm_gs<EPI_STORE>(x, w->k_in, base, ld, w->n_out, G, st);
 }
 
 // ---------------------------------------------------------------- scan
@@ -688,7 +936,7 @@ int selective_scan_forward(const void* u, const void* delta_raw, const float* de
                            int dtype, void* stream) {
   if (B < 0 || L < 0 || E <= 0 || N <= 0) return BITSSM_ERR_INVALID_ARG;
   if (dtype != BITSSM_F32 && dtype != BITSSM_BF16) return BITSSM_ERR_INVALID_ARG;
-  if (N != kScanN) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (N != kScanN || E % 8 != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (B == 0 || L == 0) {
     if (h_last != nullptr && B > 0) {
       cudaStream_t st = as_stream(stream);
@@ -729,10 +977,7 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
   if (dst == nullptr || dst_bytes < need || (reinterpret_cast<uintptr_t>(dst) & 255))
     return BITSSM_ERR_WORKSPACE;
   LayerPlan P = plan_layer(p, 1, 1, act_mode, false);
-  ExpandJobs J;
-  std::memset(&J, 0, sizeof(J));
-  fill_expand_jobs(p, P, reinterpret_cast<uint8_t*>(dst), J);
-  return launch_expand(J, act_mode == BITSSM_A16, as_stream(stream));
+  return expand_layer(p, P, reinterpret_cast<uint8_t*>(dst), as_stream(stream));
 }
 
 int bitssm_workspace_size(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
@@ -749,7 +994,10 @@ int bitssm_workspace_layout(const bitssm_layer* p, int B, int L, int dtype, int 
   if (view == nullptr) return BITSSM_ERR_INVALID_ARG;
   int rc = check_layer_args(p, B, L, dtype, act_mode);
   if (rc) return rc;
-  *view = plan_layer(p, B, L, act_mode, p->prepared != nullptr).v;
+  const LayerPlan P = plan_layer(p, B, L, act_mode, p->prepared != nullptr);
+  *view = P.v;
+  if (act_mode == BITSSM_A8 && a8_fused(P) && !(p->flags & BITSSM_KEEP_CODES))
+    view->q_x = view->q_u = view->q_y = (size_t)-1;
   return BITSSM_OK;
 }
 
@@ -776,16 +1024,16 @@ int forward_impl(const bitssm_layer* p, const void* x, void* out, const void* re
   if (prepared) {
     wexp = reinterpret_cast<const uint8_t*>(p->prepared);
   } else {
-    ExpandJobs J;
-    std::memset(&J, 0, sizeof(J));
-    fill_expand_jobs(p, P, reinterpret_cast<uint8_t*>(ws), J);
     mk.mark();
-    rc = launch_expand(J, act_mode == BITSSM_A16, st);
+    rc = expand_layer(p, P, reinterpret_cast<uint8_t*>(ws), st);
     if (rc) return rc;
     wexp = reinterpret_cast<const uint8_t*>(ws);
   }
-  rc = act_mode == BITSSM_A8 ? forward_a8(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk)
-                             : forward_a16(p, P, wexp, x, out, residual, B, L, ws, st, mk);
+  if (act_mode == BITSSM_A8)
+    rc = a8_fused(P) ? forward_a8_fused(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk)
+                     : forward_a8(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk);
+  else
+    rc = forward_a16(p, P, wexp, x, out, residual, B, L, ws, st, mk);
   if (rc == BITSSM_OK && mk.failed) rc = BITSSM_ERR_CUDA;
   return rc;
 }
@@ -803,7 +1051,9 @@ int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* 
 int bitssm_forward_launches(const bitssm_layer* p, int act_mode) {
   if (p == nullptr || (act_mode != BITSSM_A8 && act_mode != BITSSM_A16)) return -1;
   const int expand = p->prepared != nullptr ? 0 : 1;
-  return expand + (act_mode == BITSSM_A8 ? 6 : 7);
+  if (act_mode == BITSSM_A16) return expand + 7;
+  const LayerPlan P = plan_layer(p, 1, 1, act_mode, p->prepared != nullptr);
+  return expand + (a8_fused(P) ? 3 : 6);
 }
 
 int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const void* residual,

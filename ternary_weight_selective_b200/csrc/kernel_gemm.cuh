@@ -59,24 +59,14 @@ struct GemmParams {
   int ss_nparts;
   int ss_count;                // number of columns the partial sums cover
   float* r_out;                // EPI_XPROJ_A16: r_dt [M]
-};
-
-template <bool kBF16>
-struct GemmTraits {
-  static constexpr int kElemBytes = kBF16 ? 2 : 1;
-  static constexpr int kPanelElems = 128 / kElemBytes;  // K elements per 128-byte panel
-  static constexpr int kKPerMma = 32 / kElemBytes;      // K elements per MMA (32 bytes)
+  // group-scaled (W1.58A16) kernel: fp32 scales transposed, s_t[g * ld_s + n]
+  const float* s_t;
+  long ld_s;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
-}
-
-template <bool kBF16>
-__device__ __forceinline__ float acc_to_float(uint32_t bits) {
-  if constexpr (kBF16) return __uint_as_float(bits);
-  else return (float)(int)bits;  // exact: |acc| < 2^24
 }
 
 // Store 16 consecutive outputs of one row.
@@ -106,38 +96,88 @@ __device__ __forceinline__ void store16(void* base, long idx, int dtype, const f
   }
 }
 
-__device__ __forceinline__ void load16_residual(const void* base, long idx, int dtype,
-                                                float (&v)[16], int valid) {
-  if (dtype == 0) {
-    const float* p = reinterpret_cast<const float*>(base) + idx;
-    for (int j = 0; j < valid; ++j) v[j] += p[j];
-  } else {
-    const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(base) + idx;
-    for (int j = 0; j < valid; ++j) v[j] += __bfloat162float(p[j]);
-  }
-}
-
-template <bool kBF16, int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int CSPLIT>
 struct GemmConfig {
-  using Tr = GemmTraits<kBF16>;
   static constexpr int kABytes = 128 * 128;           // 128 rows x 128 B
   static constexpr int kBBytes = BN * 128;            // BN rows x 128 B
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kSmemBytes = 1024 /*align slack*/ + kBarOffset + 256;
+  static constexpr int kRedOffset = kBarOffset + 256;  // row partials [2][CSPLIT][128]
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kRedOffset + 2 * CSPLIT * 128 * 4;
   static constexpr int kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
   static constexpr int kNHalf = BN > 256 ? 2 : 1;
   static constexpr int kMmaN = BN > 256 ? 256 : BN;
+  static constexpr int kSlice = BN / CSPLIT;           // columns per epilogue warp
+  static constexpr int kThreads = 64 + 128 * CSPLIT;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 512, "BN");
   static_assert(BN <= 256 || BN == 512, "BN above 256 must be 512");
+  static_assert(kSlice % 32 == 0, "slice");
 };
 
-template <bool kBF16, int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+// Each thread of the warp reads 32 consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// 16 outputs of one row: v[j] += residual[idx + j] (vector loads when aligned).
+__device__ __forceinline__ void add_residual16(const void* base, long idx, int dtype, float (&v)[16],
+                                               int valid) {
+  if (dtype == 0) {
+    const float* p = reinterpret_cast<const float*>(base) + idx;
+    if (valid == 16 && (idx & 3) == 0) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) {
+        const float4 r = *reinterpret_cast<const float4*>(p + j);
+        v[j] += r.x; v[j + 1] += r.y; v[j + 2] += r.z; v[j + 3] += r.w;
+      }
+    } else {
+      for (int j = 0; j < valid; ++j) v[j] += p[j];
+    }
+  } else {
+    const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(base) + idx;
+    if (valid == 16 && (idx & 7) == 0) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 8) {
+        const uint4 r = *reinterpret_cast<const uint4*>(p + j);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[j + 2 * k] += __uint_as_float(w[k] << 16);
+          v[j + 2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
+        }
+      }
+    } else {
+      for (int j = 0; j < valid; ++j) v[j] += __bfloat162float(p[j]);
+    }
+  }
+}
+
+// int8 x ternary GEMM (A8).  Warp 0 lane 0: TMA producer; warp 1: TMEM
+// owner and MMA issuer (lane 0); warps 2 .. 2+4*CSPLIT-1: epilogue, warp w
+// on the 32 TMEM lanes (rows) of quadrant w % 4 and on column slice
+// (w - 2) / 4 of width BN / CSPLIT.  Row-wide reductions of the
+// whole-row epilogues are combined through shared memory.
+template <int BN, int STAGES, int EPI, int CSPLIT>
+__global__ void __launch_bounds__(GemmConfig<BN, STAGES, CSPLIT>::kThreads, 1)
     ternary_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapW, GemmParams P) {
-  using Cfg = GemmConfig<kBF16, BN, STAGES, EPI>;
-  using Tr = GemmTraits<kBF16>;
+  using Cfg = GemmConfig<BN, STAGES, CSPLIT>;
+  constexpr int kPanelElems = 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -147,12 +187,14 @@ __global__ void __launch_bounds__(192, 1)
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   const uint32_t done_bar = bar_base + 8u * (2 * STAGES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kBarOffset + 8 * (2 * STAGES + 1));
+  float* red_a = reinterpret_cast<float*>(smem + Cfg::kRedOffset);  // [CSPLIT][128]
+  float* red_b = red_a + CSPLIT * 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128;
   const int n0 = blockIdx.y * BN;
-  const int num_panels = (P.K + Tr::kPanelElems - 1) / Tr::kPanelElems;
+  const int num_panels = (P.K + kPanelElems - 1) / kPanelElems;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -183,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
       if (p >= STAGES && !mbar_wait(empty_bar(s), ph ^ 1u, DEVFLAG_TIMEOUT_TMA)) break;
       const uint32_t sa = sbase + s * Cfg::kStageBytes;
       mbar_arrive_expect_tx(full_bar(s), kTx);
-      const int kc = p * Tr::kPanelElems;
+      const int kc = p * kPanelElems;
       tma_load_2d(sa, &mapA, kc, m0, full_bar(s));
 #pragma unroll
       for (int h = 0; h < BN / kWBox; ++h)
@@ -191,8 +233,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t kIdesc =
-        kBF16 ? umma_idesc(1u, 1u, 128u, (uint32_t)Cfg::kMmaN) : umma_idesc(2u, 1u, 128u, (uint32_t)Cfg::kMmaN);
+    constexpr uint32_t kIdesc = umma_idesc(2u, 1u, 128u, (uint32_t)Cfg::kMmaN);
     bool ok = true;
     for (int p = 0; p < num_panels && ok; ++p) {
       const int s = p % STAGES;
@@ -208,9 +249,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int h = 0; h < Cfg::kNHalf; ++h) {
           const uint64_t bdesc = sw128_kmajor_desc(sb + h * 256 * 128 + kk * 32);
-          const uint32_t acc = (p > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (kBF16) umma_bf16(tmem + h * 256, adesc, bdesc, kIdesc, acc);
-          else umma_i8(tmem + h * 256, adesc, bdesc, kIdesc, acc);
+          umma_i8(tmem + h * 256, adesc, bdesc, kIdesc, (p > 0 || kk > 0) ? 1u : 0u);
         }
       }
       umma_commit(empty_bar(s));
@@ -219,120 +258,176 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int q = warp & 3;
+    const int slice = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const int m = m0 + row;
     const bool live = m < P.M;
-    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    const int cs = slice * Cfg::kSlice;  // first column of this warp's slice
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + cs;
     const bool ok = mbar_wait(done_bar, 0u, DEVFLAG_TIMEOUT_EPI);
     tc_fence_after();
-    if (ok) {
-      const float rs = (P.row_scale != nullptr && live) ? P.row_scale[m] : 1.0f;
+    const float rs = (P.row_scale != nullptr && live) ? P.row_scale[m] : 1.0f;
 
-      if constexpr (EPI == EPI_STORE) {
-        const float f = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;
-        const int ncols = min(BN, P.N - n0);
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
-          if (!live || c0 >= ncols) continue;
-          const int valid = min(16, ncols - c0);
-          const long idx = (long)m * P.ld_out + n0 + c0;
+    if constexpr (EPI == EPI_STORE) {
+      const float f = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;
+      const int ncols = min(BN, P.N - n0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
+        if (!ok || !live) continue;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int col = cs + c0 + hh * 16;
+          if (col >= ncols) break;
+          const int valid = min(16, ncols - col);
+          const long idx = (long)m * P.ld_out + n0 + col;
           if (P.out_dtype == 2) {
             int* o = reinterpret_cast<int*>(P.out) + idx;
-            for (int j = 0; j < valid; ++j) o[j] = (int)r[j];
+            for (int j = 0; j < valid; ++j) o[j] = (int)r[hh * 16 + j];
             continue;
           }
           float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = acc_to_float<kBF16>(r[j]) * f;
-          if (P.residual != nullptr) load16_residual(P.residual, idx, P.out_dtype, v, valid);
+          for (int j = 0; j < 16; ++j) v[j] = i2f_exact((int)r[hh * 16 + j]) * f;
+          if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
           store16(P.out, idx, P.out_dtype, v, valid);
         }
-      } else if constexpr (EPI == EPI_QUANT_ROW) {
-        // whole row in this tile (n0 == 0, N <= BN)
-        const int N = P.N;
-        int maxabs = 0;
-        float ss = 0.f;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
+      }
+    } else if constexpr (EPI == EPI_QUANT_ROW) {
+      // whole row in this tile (n0 == 0, N <= BN).  Pass 1: max|acc| in
+      // integers; pass 2: u = acc * c, the codes of the int32 row and
+      // sum(acc^2); the slices of a row combine both through shared memory.
+      const int N = P.N;
+      const bool full = N == BN;
+      int maxabs = 0;
+#pragma unroll 1
+      for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c0 + j < N) {
-              const int a = (int)r[j];
-              maxabs = max(maxabs, abs(a));
-              const float fa = (float)a;
-              ss = fmaf(fa, fa, ss);
-            }
-          }
+        for (int j = 0; j < 32; ++j)
+          if (full || cs + c0 + j < N) maxabs = max(maxabs, abs((int)r[j]));
+      }
+      if constexpr (CSPLIT > 1) {
+        red_a[slice * 128 + row] = __int_as_float(maxabs);
+        named_bar_sync(1, 128 * CSPLIT);
+#pragma unroll
+        for (int k = 0; k < CSPLIT; ++k) maxabs = max(maxabs, __float_as_int(red_a[k * 128 + row]));
+      }
+      const float c = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;  // u = acc * c
+      const float sigma = maxabs > 0 ? __fdiv_rn(127.f, (float)maxabs) : 0.f;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
+        const int col0 = cs + c0;
+        float a[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          a[j] = i2f_exact((int)r[j]);
+          if (full || col0 + j < N) ss = fmaf(a[j], a[j], ss);
         }
-        const float c = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;  // u = acc * c
-        const float sigma = maxabs > 0 ? __fdiv_rn(127.f, (float)maxabs) : 0.f;
-        if (live) {
-          const float mu = (float)maxabs * c;
-          const float r_u = 1.0f / sqrtf(c * c * (ss / (float)N) + kEpsNorm);
-          P.deq_out[m] = mu * r_u / 127.f;
-        }
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
-          if (!live) continue;
-          const int valid = min(16, N - c0);
+        if (!ok || !live) continue;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int col = col0 + hh * 16;
+          const int valid = full ? 16 : min(16, N - col);
           if (valid > 0) {
             float v[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = (float)(int)r[j] * c;
-            store16(P.out, (long)m * P.ld_out + c0, 0, v, valid);
+            for (int j = 0; j < 16; ++j) v[j] = a[hh * 16 + j] * c;
+            store16(P.out, (long)m * P.ld_out + col, 0, v, valid);
           }
-          if (c0 < P.ld_q) {
+          if (col < P.ld_q) {
             uint32_t w[4];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              uint32_t word = 0;
+            for (int k = 0; k < 4; ++k) {
+              uint32_t cb[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const int col = c0 + g * 4 + j;
-                const int code = col < N ? quant_code((float)(int)r[g * 4 + j], sigma) : 0;
-                word |= (uint32_t)(code & 0xff) << (8 * j);
+                const int jj = hh * 16 + 4 * k + j;
+                cb[j] = (full || col0 + jj < N) ? code_bits(a[jj], sigma) : 0u;
               }
-              w[g] = word;
+              w[k] = pack4(cb[0], cb[1], cb[2], cb[3]);
             }
-            *reinterpret_cast<uint4*>(P.q_out + (long)m * P.ld_q + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(P.q_out + (long)m * P.ld_q + col) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-      } else if constexpr (EPI == EPI_XPROJ_A8) {
-        // columns: [0,R) dt | [R,R+Ns) B | [R+Ns,R+2Ns) C ; whole row in this tile
-        const int R = P.R, Ns = P.Ns;
-        int maxabs = 0;
-        float ss = 0.f;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
+      }
+      if constexpr (CSPLIT > 1) {
+        red_b[slice * 128 + row] = ss;
+        named_bar_sync(1, 128 * CSPLIT);
+        ss = 0.f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = c0 + j;
+        for (int k = 0; k < CSPLIT; ++k) ss += red_b[k * 128 + row];
+      }
+      if (live && slice == 0) {
+        const float mu = (float)maxabs * c;
+        const float r_u = 1.0f / sqrtf(c * c * (ss / (float)N) + kEpsNorm);
+        P.deq_out[m] = mu * r_u / 127.f;
+      }
+    } else if constexpr (EPI == EPI_XPROJ_A8) {
+      // columns: [0,R) dt | [R,R+Ns) B | [R+Ns,R+2Ns) C ; one slice holds the whole row
+      static_assert(CSPLIT == 1, "x_proj epilogue keeps the whole row in one warp");
+      const int R = P.R, Ns = P.Ns;
+      int maxabs = 0;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN && c0 < R; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (c0 + j < R) {
+            const int a = (int)r[j];
+            maxabs = max(maxabs, abs(a));
+            const float fa = i2f_exact(a);
+            ss = fmaf(fa, fa, ss);
+          }
+        }
+      }
+      const float cdt = *P.alpha_dt * rs;  // dt_low = acc * cdt
+      const float sigma = maxabs > 0 ? __fdiv_rn(127.f, (float)maxabs) : 0.f;
+      if (live) {
+        const float mdt = (float)maxabs * cdt;
+        const float r_dt = 1.0f / sqrtf(cdt * cdt * (ss / (float)R) + kEpsNorm);
+        P.deq_out[m] = mdt * r_dt / 127.f;
+      }
+      const float cB = *P.alpha_B * rs, cC = *P.alpha_C * rs;
+      const bool fast = (R % 16 == 0) && (Ns == 16) && (P.ld_q == R);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
+        if (!ok || !live) continue;
+        if (fast) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int col = c0 + hh * 16;
+            const uint32_t* rr = r + hh * 16;
             if (col < R) {
-              const int a = (int)r[j];
-              maxabs = max(maxabs, abs(a));
-              const float fa = (float)a;
-              ss = fmaf(fa, fa, ss);
+              uint32_t w[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                w[k] = pack4(code_bits(i2f_exact((int)rr[4 * k]), sigma),
+                             code_bits(i2f_exact((int)rr[4 * k + 1]), sigma),
+                             code_bits(i2f_exact((int)rr[4 * k + 2]), sigma),
+                             code_bits(i2f_exact((int)rr[4 * k + 3]), sigma));
+              *reinterpret_cast<uint4*>(P.q_out + (long)m * P.ld_q + col) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else if (col < R + 2 * Ns) {
+              const bool isB = col < R + Ns;
+              const float cf = isB ? cB : cC;
+              float4* dst = reinterpret_cast<float4*>((isB ? P.Bm : P.Cm) + (long)m * Ns);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_float4(i2f_exact((int)rr[4 * v]) * cf, i2f_exact((int)rr[4 * v + 1]) * cf,
+                                     i2f_exact((int)rr[4 * v + 2]) * cf, i2f_exact((int)rr[4 * v + 3]) * cf);
             }
           }
-        }
-        const float cdt = *P.alpha_dt * rs;  // dt_low = acc * cdt
-        const float sigma = maxabs > 0 ? __fdiv_rn(127.f, (float)maxabs) : 0.f;
-        if (live) {
-          const float mdt = (float)maxabs * cdt;
-          const float r_dt = 1.0f / sqrtf(cdt * cdt * (ss / (float)R) + kEpsNorm);
-          P.deq_out[m] = mdt * r_dt / 127.f;
-        }
-        const float cB = *P.alpha_B * rs, cC = *P.alpha_C * rs;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
-          if (!live) continue;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
+        } else {
+          for (int j = 0; j < 32; ++j) {
             const int col = c0 + j;
             const int a = (int)r[j];
             if (col < R) {
@@ -344,56 +439,9 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
-        if (live)
-          for (int col = R; col < P.ld_q; ++col) P.q_out[(long)m * P.ld_q + col] = 0;
-      } else if constexpr (EPI == EPI_ROWSS) {
-        const int ncols = min(BN, P.N - n0);
-        float ss = 0.f;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
-          if (!live || c0 >= ncols) continue;
-          const int valid = min(16, ncols - c0);
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v[j] = __uint_as_float(r[j]) * rs;
-            if (j < valid) ss = fmaf(v[j], v[j], ss);
-          }
-          store16(P.out, (long)m * P.ld_out + n0 + c0, 1, v, valid);
-        }
-        if (live) P.ss_part[(long)m * gridDim.y + blockIdx.y] = ss;
-      } else if constexpr (EPI == EPI_XPROJ_A16) {
-        const int R = P.R, Ns = P.Ns;
-        float r_u = 1.f;
-        if (live) {
-          float t = 0.f;
-          for (int j = 0; j < P.ss_nparts; ++j) t += P.ss_in[(long)m * P.ss_nparts + j];
-          r_u = 1.0f / sqrtf(t / (float)P.ss_count + kEpsNorm);
-        }
-        float ss = 0.f;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(trow + c0, r);
-          if (!live) continue;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = c0 + j;
-            const float v = __uint_as_float(r[j]) * r_u;
-            if (col < R) {
-              const __nv_bfloat16 b = __float2bfloat16_rn(v);
-              reinterpret_cast<__nv_bfloat16*>(P.out)[(long)m * P.ld_out + col] = b;
-              const float vb = __bfloat162float(b);
-              ss = fmaf(vb, vb, ss);
-            } else if (col < R + Ns) {
-              P.Bm[(long)m * Ns + (col - R)] = v;
-            } else if (col < R + 2 * Ns) {
-              P.Cm[(long)m * Ns + (col - R - Ns)] = v;
-            }
-          }
-        }
-        if (live) P.r_out[m] = 1.0f / sqrtf(ss / (float)R + kEpsNorm);
       }
+      if (live && !fast)
+        for (int col = R; col < P.ld_q; ++col) P.q_out[(long)m * P.ld_q + col] = 0;
     }
   }
 
@@ -402,6 +450,227 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// W1.58A16 GEMM with exact per-group weight scales ("Ternary Mamba: Grouped
+// Quantization-Aware Training of W1.58A16 State Space Models", abstract):
+//
+//   D[m, n] = sum_g s[n, g] * sum_{k in group g} x[m, k] * w[n, k]
+//
+// The tensor core multiplies bf16 activations by exact ternary weights
+// {-1, 0, 1} and accumulates one 128-wide K group at a time into one of two
+// TMEM buffers (cols 0..BN-1 and 256..256+BN-1).  Eight epilogue warps (two
+// per TMEM lane quadrant, each owning BN/2 columns) read the finished group
+// from TMEM, multiply it by the fp32 group scales and add it to fp32
+// register accumulators, while the MMA warp fills the other buffer with the
+// next group.  The scale is thus applied in fp32 exactly as defined, not
+// rounded into the bf16 operand.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <int BN, int STAGES>
+struct GsConfig {
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
+  static constexpr int kHalf = BN / 2;  // columns per epilogue warp
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(320, 1)
+    ternary_gemm_gs_kernel(const __grid_constant__ CUtensorMap mapA,
+                           const __grid_constant__ CUtensorMap mapW, GemmParams P) {
+  using Cfg = GsConfig<BN, STAGES>;
+  constexpr int kPanel = 64;             // bf16 elements per 128-byte panel
+  constexpr int kPanelsPerGroup = 2;     // 128-element weight groups
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_base = sbase + Cfg::kBarOffset;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto pfull_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + b); };
+  auto pempty_bar = [&](int b) { return bar_base + 8u * (2 * STAGES + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kBarOffset + 8 * (2 * STAGES + 4));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128;
+  const int n0 = blockIdx.y * BN;
+  const int num_panels = (P.K + kPanel - 1) / kPanel;
+  const int num_groups = (num_panels + kPanelsPerGroup - 1) / kPanelsPerGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(pfull_bar(b), 1);
+      mbar_init(pempty_bar(b), 8);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    constexpr uint32_t kTx = Cfg::kABytes + Cfg::kBBytes;
+    for (int p = 0; p < num_panels; ++p) {
+      const int s = p % STAGES;
+      const uint32_t ph = (uint32_t)(p / STAGES) & 1u;
+      if (p >= STAGES && !mbar_wait(empty_bar(s), ph ^ 1u, DEVFLAG_TIMEOUT_TMA)) break;
+      const uint32_t sa = sbase + s * Cfg::kStageBytes;
+      mbar_arrive_expect_tx(full_bar(s), kTx);
+      const int kc = p * kPanel;
+      tma_load_2d(sa, &mapA, kc, m0, full_bar(s));
+      tma_load_2d(sa + Cfg::kABytes, &mapW, kc, n0, full_bar(s));
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t kIdesc = umma_idesc(1u, 1u, 128u, (uint32_t)BN);
+    bool ok = true;
+    int p = 0;
+    for (int g = 0; g < num_groups && ok; ++g) {
+      const int buf = g & 1;
+      if (g >= 2) ok = mbar_wait(pempty_bar(buf), (uint32_t)((g >> 1) - 1) & 1u, DEVFLAG_TIMEOUT_MMA);
+      if (!ok) break;
+      tc_fence_after();
+      const int p_end = min(num_panels, p + kPanelsPerGroup);
+      for (int pi = 0; p < p_end; ++p, ++pi) {
+        const int s = p % STAGES;
+        const uint32_t ph = (uint32_t)(p / STAGES) & 1u;
+        ok = mbar_wait(full_bar(s), ph, DEVFLAG_TIMEOUT_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sa = sbase + s * Cfg::kStageBytes;
+        const uint32_t sb = sa + Cfg::kABytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adesc = sw128_kmajor_desc(sa + kk * 32);
+          const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
+          umma_bf16(tmem + buf * 256, adesc, bdesc, kIdesc, (pi > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(empty_bar(s));
+      }
+      umma_commit(pfull_bar(buf));
+    }
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const int m = m0 + row;
+    const bool live = m < P.M;
+    const int c_base = half * Cfg::kHalf;  // first column of this warp (tile-relative)
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + c_base;
+    float acc[Cfg::kHalf];
+#pragma unroll
+    for (int j = 0; j < Cfg::kHalf; ++j) acc[j] = 0.f;
+    bool ok = true;
+    for (int g = 0; g < num_groups; ++g) {
+      const int buf = g & 1;
+      ok = mbar_wait(pfull_bar(buf), (uint32_t)(g >> 1) & 1u, DEVFLAG_TIMEOUT_EPI);
+      if (!ok) break;
+      tc_fence_after();
+      const float* sg = P.s_t + (long)g * P.ld_s + n0 + c_base;
+#pragma unroll
+      for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(trow + buf * 256 + c0, r);
+        const float4* s4 = reinterpret_cast<const float4*>(sg + c0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 sv = __ldg(s4 + v);
+          acc[c0 + 4 * v + 0] = fmaf(sv.x, __uint_as_float(r[4 * v + 0]), acc[c0 + 4 * v + 0]);
+          acc[c0 + 4 * v + 1] = fmaf(sv.y, __uint_as_float(r[4 * v + 1]), acc[c0 + 4 * v + 1]);
+          acc[c0 + 4 * v + 2] = fmaf(sv.z, __uint_as_float(r[4 * v + 2]), acc[c0 + 4 * v + 2]);
+          acc[c0 + 4 * v + 3] = fmaf(sv.w, __uint_as_float(r[4 * v + 3]), acc[c0 + 4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pempty_bar(buf));
+    }
+    if (ok && live) {
+      const float rs = P.row_scale != nullptr ? P.row_scale[m] : 1.0f;
+      if constexpr (EPI == EPI_STORE) {
+        const int ncols = min(BN, P.N - n0);
+#pragma unroll
+        for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
+          const int col = c_base + c0;
+          if (col >= ncols) break;
+          const int valid = min(16, ncols - col);
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = acc[c0 + j] * rs;
+          const long idx = (long)m * P.ld_out + n0 + col;
+          if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
+          store16(P.out, idx, P.out_dtype, v, valid);
+        }
+      } else if constexpr (EPI == EPI_ROWSS) {
+        const int ncols = min(BN, P.N - n0);
+        float ss = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
+          const int col = c_base + c0;
+          if (col >= ncols) break;
+          const int valid = min(16, ncols - col);
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v[j] = acc[c0 + j] * rs;
+            if (j < valid) ss = fmaf(v[j], v[j], ss);
+          }
+          store16(P.out, (long)m * P.ld_out + n0 + col, 1, v, valid);
+        }
+        P.ss_part[(long)m * (2 * gridDim.y) + 2 * blockIdx.y + half] = ss;
+      } else if constexpr (EPI == EPI_XPROJ_A16) {
+        // columns [0,R) dt (all in half 0: R <= BN/2) | [R,R+Ns) B | [R+Ns,R+2Ns) C
+        const int R = P.R, Ns = P.Ns;
+        float t = 0.f;
+        for (int j = 0; j < P.ss_nparts; ++j) t += P.ss_in[(long)m * P.ss_nparts + j];
+        const float r_u = 1.0f / sqrtf(t / (float)P.ss_count + kEpsNorm);
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < Cfg::kHalf; ++j) {
+          const int col = c_base + j;
+          const float v = acc[j] * r_u;
+          if (col < R) {
+            const __nv_bfloat16 b = __float2bfloat16_rn(v);
+            reinterpret_cast<__nv_bfloat16*>(P.out)[(long)m * P.ld_out + col] = b;
+            const float vb = __bfloat162float(b);
+            ss = fmaf(vb, vb, ss);
+          } else if (col < R + Ns) {
+            P.Bm[(long)m * Ns + (col - R)] = v;
+          } else if (col < R + 2 * Ns) {
+            P.Cm[(long)m * Ns + (col - R - Ns)] = v;
+          }
+        }
+        if (half == 0) P.r_out[m] = 1.0f / sqrtf(ss / (float)R + kEpsNorm);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 

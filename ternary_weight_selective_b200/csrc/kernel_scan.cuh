@@ -9,10 +9,8 @@
 // Parallel structure: the recurrence is an associative composition of affine
 // maps h -> a h + b per (batch, channel, state); the B*E*16 state lanes are
 // independent, and a step of one lane depends on the previous step only
-// through one FMA (a and b are computed off the chain).  This kernel gives
-// every (batch, channel) 16/NPT threads, each owning NPT states in
-// registers, walks the time axis in chunks of TC steps staged in shared
-// memory, and reduces y over the channel's threads with warp shuffles.
+// through one FMA (a and b are computed off the chain), so the B*E*16 lanes
+// are scanned side by side, each walking the time axis once.
 //
 // FUSED_DT: delta_raw is not read from memory but formed here from the int8
 // codes of the low-rank Delta projection (the Delta-up BitLinear):
@@ -29,7 +27,6 @@
 namespace bitssm {
 
 constexpr int kScanN = 16;   // d_state
-constexpr int kScanTC = 32;  // time steps per staged chunk
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanParams {
@@ -41,7 +38,7 @@ struct ScanParams {
   const int8_t* W_up;     // [E, ld_w] int8 {-1,0,1} (fused)
   long ld_w;
   const float* s_up;      // device scalar (fused)
-  int R;                  // padded to a multiple of 4 (zero codes beyond dt_rank)
+  int R;                  // padded to a multiple of 16 (zero codes beyond dt_rank)
   const float* bias;      // [E]
   const float* A;         // [E, 16]
   const float* Bm;        // [B, L, 16]
@@ -62,50 +59,160 @@ __device__ __forceinline__ void store_as<__nv_bfloat16>(__nv_bfloat16* p, float 
   *p = __float2bfloat16_rn(v);
 }
 
-__device__ __forceinline__ float softplus_f(float z) {
-  return fmaxf(z, 0.f) + log1pf(expf(-fabsf(z)));
+// softplus(z) = max(z, 0) + log1p(t), t = exp(-|z|) in (0, 1], with log1p(t)
+// = t * p(t) and p a degree-8 least-squares fit of log1p(t)/t on [0, 1]
+// (coefficients from gen_softplus_poly.py; relative error ~3e-8 before
+// float32 rounding).  One exp2 and nine FMAs.
+__device__ __forceinline__ float softplus_fast(float z) {
+  const float t = ex2_approx(-fabsf(z) * kLog2e);
+  float p = 5.253457797e-03f;
+  p = fmaf(p, t, -2.958850739e-02f);
+  p = fmaf(p, t, 7.836166802e-02f);
+  p = fmaf(p, t, -1.367476971e-01f);
+  p = fmaf(p, t, 1.911143108e-01f);
+  p = fmaf(p, t, -2.484436989e-01f);
+  p = fmaf(p, t, 3.331927134e-01f);
+  p = fmaf(p, t, -4.999950152e-01f);
+  p = fmaf(p, t, 9.999999705e-01f);
+  return fmaxf(z, 0.f) + t * p;
 }
 
-// Shared-memory footprint of one CTA (bytes), for CE channels per CTA.
-__host__ __device__ constexpr int scan_smem_bytes(int CE, int Rmax) {
-  return kScanTC * CE * 4 * 3        // u_s, dt_s, y_s
-         + kScanTC * kScanN * 4 * 2  // B_s, C_s
-         + kScanTC * Rmax            // qdt_s
-         + kScanTC * 4               // deq_s
-         + CE * Rmax;                // W_s
+// Sum over the TPC threads of a channel of yp[s] (one partial per step s of
+// the block), scattered so that thread g of the channel returns the total
+// for step g: log2(TPC) rounds of pairwise exchange, halving the kept steps.
+template <int TPC>
+__device__ __forceinline__ float reduce_scatter(const float (&yp)[TPC], int g);
+template <>
+__device__ __forceinline__ float reduce_scatter<1>(const float (&yp)[1], int) { return yp[0]; }
+template <>
+__device__ __forceinline__ float reduce_scatter<2>(const float (&yp)[2], int g) {
+  const bool b0 = g & 1;
+  float keep = b0 ? yp[1] : yp[0];
+  const float send = b0 ? yp[0] : yp[1];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+template <>
+__device__ __forceinline__ float reduce_scatter<4>(const float (&yp)[4], int g) {
+  const bool b1 = (g >> 1) & 1;
+  float k0 = b1 ? yp[2] : yp[0];
+  float k1 = b1 ? yp[3] : yp[1];
+  const float s0 = b1 ? yp[0] : yp[2];
+  const float s1 = b1 ? yp[1] : yp[3];
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+  const bool b0 = g & 1;
+  float keep = b0 ? k1 : k0;
+  const float send = b0 ? k0 : k1;
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
-template <int NPT, bool FUSED, typename Tu, typename Td, typename Ty>
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+constexpr int kScanChunk = 16;  // time steps per staged chunk
+
+// Shared-memory layout of one stage (one chunk of kScanChunk steps).
+template <int CE, bool FUSED, typename Tu, typename Td>
+struct ScanStage {
+  static constexpr int kU = kScanChunk * CE * (int)sizeof(Tu);
+  static constexpr int kD = FUSED ? 0 : kScanChunk * CE * (int)sizeof(Td);
+  static constexpr int kBC = kScanChunk * kScanN * 4;
+  static constexpr int kQ = FUSED ? kScanChunk * 128 : 0;  // dt codes, row pitch 128 B
+  static constexpr int kDeq = FUSED ? kScanChunk * 4 : 0;
+  static constexpr int oU = 0, oD = oU + kU, oB = oD + kD, oC = oB + kBC, oQ = oC + kBC,
+                       oDeq = oQ + kQ;
+  static constexpr int kBytes = oDeq + kDeq;
+};
+
+// Selective scan.  A CTA of 128 threads owns CE = 128*NPT/16 channels of one
+// batch; each channel has TPC = 16/NPT consecutive lanes, lane g owning
+// states g*NPT .. g*NPT+NPT-1 in registers.  Inputs are staged in chunks of
+// 16 steps through a double-buffered shared-memory ring filled with cp.async
+// (the copy of chunk c+1 runs while chunk c is computed; one barrier per
+// chunk).  Per chunk, lane g first forms delta, delta*u and D*u for its
+// 16/TPC steps (t = g, g+TPC, ...; the Delta-up dot product and the softplus
+// are computed once per (token, channel), and the independent steps give
+// the scheduler room to overlap them); then the 16 steps are advanced, fully
+// unrolled, with the channel's lanes exchanging delta and delta*u by
+// shuffles, and the per-step partial outputs are reduce-scattered so that
+// lane g stores y for its own steps.  RV = number of 16-code vectors of the
+// Delta-up row (dt_rank padded to 16*RV).
+template <int NPT, bool FUSED, int RV, typename Tu, typename Td, typename Ty>
 __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
-  constexpr int TPC = kScanN / NPT;  // threads per channel
-  constexpr int CE = 128 / TPC;      // channels per CTA
+  constexpr int TPC = kScanN / NPT;
+  constexpr int CE = 128 / TPC;
+  constexpr int SPL = kScanChunk / TPC;  // steps per lane per chunk
+  using St = ScanStage<CE, FUSED, Tu, Td>;
   extern __shared__ __align__(16) uint8_t smem[];
-  float* u_s = reinterpret_cast<float*>(smem);
-  float* dt_s = u_s + kScanTC * CE;
-  float* y_s = dt_s + kScanTC * CE;
-  float* B_s = y_s + kScanTC * CE;
-  float* C_s = B_s + kScanTC * kScanN;
-  float* deq_s = C_s + kScanTC * kScanN;
-  int8_t* qdt_s = reinterpret_cast<int8_t*>(deq_s + kScanTC);
-  int8_t* W_s = qdt_s + kScanTC * (FUSED ? P.R : 0);
+  const uint32_t sbase = smem_u32(smem);
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const int b = blockIdx.y;
   const int e0 = blockIdx.x * CE;
-  const int c = tid / TPC;        // channel within the CTA
-  const int g = tid % TPC;        // state group
+  const int c = tid / TPC;
+  const int g = tid % TPC;
   const int e = e0 + c;
   const bool ch_ok = e < P.E;
   const int E = P.E, L = P.L;
   const long tok0 = (long)b * L;
+  const int src0 = lane & ~(TPC - 1);
 
-  if constexpr (FUSED) {
-    // Delta-up weights of this CTA's channels, [CE][R]
-    for (int i = tid; i < CE * P.R; i += 128) {
-      const int cc = i / P.R, r = i - cc * P.R;
-      W_s[i] = (e0 + cc < E) ? P.W_up[(long)(e0 + cc) * P.ld_w + r] : (int8_t)0;
+  // issue the copies of chunk `ch` into stage `stg`
+  auto issue = [&](int ch, int stg) {
+    const int t0 = ch * kScanChunk;
+    const uint32_t sb = sbase + stg * St::kBytes;
+    constexpr int kVecRow = CE * (int)sizeof(Tu) / 16;  // 16-byte vectors per step row
+    for (int i = tid; i < kScanChunk * kVecRow; i += 128) {
+      const int t = i / kVecRow, v = i - t * kVecRow;
+      const int ee = e0 + v * (16 / (int)sizeof(Tu));
+      const int avail = (t0 + t < L) ? max(0, min(16, (E - ee) * (int)sizeof(Tu))) : 0;
+      const Tu* src = reinterpret_cast<const Tu*>(P.u) + (tok0 + min(t0 + t, L - 1)) * E + min(ee, E - 1);
+      cp_async16(sb + St::oU + i * 16, src, avail);
     }
-  }
+    if constexpr (!FUSED) {
+      constexpr int kVecRowD = CE * (int)sizeof(Td) / 16;
+      for (int i = tid; i < kScanChunk * kVecRowD; i += 128) {
+        const int t = i / kVecRowD, v = i - t * kVecRowD;
+        const int ee = e0 + v * (16 / (int)sizeof(Td));
+        const int avail = (t0 + t < L) ? max(0, min(16, (E - ee) * (int)sizeof(Td))) : 0;
+        const Td* src = reinterpret_cast<const Td*>(P.delta_raw) + (tok0 + min(t0 + t, L - 1)) * E + min(ee, E - 1);
+        cp_async16(sb + St::oD + i * 16, src, avail);
+      }
+    }
+    // B and C: kScanChunk rows of 64 bytes each, contiguous
+    for (int i = tid; i < kScanChunk * 4 * 2; i += 128) {
+      const int which = i / (kScanChunk * 4), j = i - which * (kScanChunk * 4);
+      const int t = j / 4;
+      const float* base = which ? P.Cm : P.Bm;
+      const int avail = (t0 + t < L) ? 16 : 0;
+      cp_async16(sb + (which ? St::oC : St::oB) + j * 16,
+                 base + (tok0 + min(t0 + t, L - 1)) * kScanN + (j & 3) * 4, avail);
+    }
+    if constexpr (FUSED) {
+      for (int i = tid; i < kScanChunk * RV; i += 128) {
+        const int t = i / RV, v = i - t * RV;
+        const int avail = (t0 + t < L) ? 16 : 0;
+        cp_async16(sb + St::oQ + t * 128 + v * 16,
+                   P.q_dt + (tok0 + min(t0 + t, L - 1)) * P.ld_qdt + v * 16, avail);
+      }
+      for (int t = tid; t < kScanChunk; t += 128)
+        cp_async4(sb + St::oDeq + t * 4, P.deq_dt + tok0 + min(t0 + t, L - 1), (t0 + t < L) ? 4 : 0);
+    }
+  };
 
   float A2[NPT], h[NPT];
 #pragma unroll
@@ -115,78 +222,112 @@ __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
     h[j] = (ch_ok && P.h0 != nullptr) ? P.h0[((long)b * E + e) * kScanN + n] : 0.f;
   }
   const float Dv = ch_ok ? P.D[e] : 0.f;
+  const float bias = ch_ok ? P.bias[e] : 0.f;
   float s_up = 0.f;
-  if constexpr (FUSED) s_up = *P.s_up;
+  int4 wq[FUSED ? RV : 1];
+  if constexpr (FUSED) {
+    s_up = *P.s_up;
+#pragma unroll
+    for (int r = 0; r < RV; ++r)
+      wq[r] = ch_ok ? __ldg(reinterpret_cast<const int4*>(P.W_up + (long)e * P.ld_w) + r)
+                    : make_int4(0, 0, 0, 0);
+  }
+  Ty* yrow = reinterpret_cast<Ty*>(P.y) + tok0 * E + e;
 
-  for (int t0 = 0; t0 < L; t0 += kScanTC) {
-    const int tc = min(kScanTC, L - t0);
-    __syncthreads();  // previous chunk's y_s consumed, W_s written
-    // ---- stage the chunk
-    for (int i = tid; i < kScanTC * CE; i += 128) {
-      const int t = i / CE, cc = i - t * CE;
-      float uv = 0.f, dv = 0.f;
-      if (t < tc && e0 + cc < E) {
-        const long idx = (tok0 + t0 + t) * E + e0 + cc;
-        uv = load_as_float(reinterpret_cast<const Tu*>(P.u) + idx);
-        if constexpr (!FUSED) dv = load_as_float(reinterpret_cast<const Td*>(P.delta_raw) + idx);
-      }
-      u_s[i] = uv;
-      dt_s[i] = dv;
-    }
-    for (int i = tid; i < kScanTC * kScanN; i += 128) {
-      const int t = i / kScanN;
-      const long idx = (tok0 + t0) * kScanN + i;
-      B_s[i] = t < tc ? P.Bm[idx] : 0.f;
-      C_s[i] = t < tc ? P.Cm[idx] : 0.f;
-    }
-    if constexpr (FUSED) {
-      for (int i = tid; i < kScanTC * P.R; i += 128) {
-        const int t = i / P.R, r = i - t * P.R;
-        qdt_s[i] = t < tc ? P.q_dt[(tok0 + t0 + t) * P.ld_qdt + r] : (int8_t)0;
-      }
-      for (int t = tid; t < kScanTC; t += 128) deq_s[t] = t < tc ? P.deq_dt[tok0 + t0 + t] : 0.f;
-    }
-    __syncthreads();
-    // ---- phase A: delta for every (t, channel) of the chunk, once
-    for (int i = tid; i < kScanTC * CE; i += 128) {
-      const int t = i / CE, cc = i - t * CE;
+  const int nchunks = (L + kScanChunk - 1) / kScanChunk;
+  issue(0, 0);
+  cp_async_commit();
+  for (int ch = 0; ch < nchunks; ++ch) {
+    cp_async_wait_all();
+    __syncthreads();  // chunk ch is visible; chunk ch-1's stage is free
+    if (ch + 1 < nchunks) issue(ch + 1, (ch + 1) & 1);
+    cp_async_commit();
+    const uint8_t* sp = smem + (ch & 1) * St::kBytes;
+    const Tu* u_s = reinterpret_cast<const Tu*>(sp + St::oU);
+    const float* B_s = reinterpret_cast<const float*>(sp + St::oB);
+    const float* C_s = reinterpret_cast<const float*>(sp + St::oC);
+    const int t0 = ch * kScanChunk;
+    const int steps = min(kScanChunk, L - t0);
+
+    // ---- delta, delta*u and D*u of this lane's steps tl = i*TPC + g
+    float dl[SPL], du[SPL], Du[SPL];
+#pragma unroll
+    for (int i = 0; i < SPL; ++i) {
+      const int tl = i * TPC + g;
+      const float uv = load_as_float(u_s + tl * CE + c);
       float z;
       if constexpr (FUSED) {
+        const int4* qv = reinterpret_cast<const int4*>(sp + St::oQ + tl * 128);
         int acc = 0;
-        const int* wq = reinterpret_cast<const int*>(W_s + cc * P.R);
-        const int* qq = reinterpret_cast<const int*>(qdt_s + t * P.R);
-        for (int r4 = 0; r4 < P.R / 4; ++r4) acc = __dp4a(wq[r4], qq[r4], acc);
-        z = (float)acc * s_up * deq_s[t];
+#pragma unroll
+        for (int r = 0; r < RV; ++r) {
+          const int4 q4 = qv[r];
+          acc = __dp4a(wq[r].x, q4.x, acc);
+          acc = __dp4a(wq[r].y, q4.y, acc);
+          acc = __dp4a(wq[r].z, q4.z, acc);
+          acc = __dp4a(wq[r].w, q4.w, acc);
+        }
+        z = fmaf((float)acc * s_up, reinterpret_cast<const float*>(sp + St::oDeq)[tl], bias);
       } else {
-        z = dt_s[i];
+        z = load_as_float(reinterpret_cast<const Td*>(sp + St::oD) + tl * CE + c) + bias;
       }
-      const float bias = (e0 + cc < E) ? P.bias[e0 + cc] : 0.f;
-      dt_s[i] = softplus_f(z + bias);
+      dl[i] = tl < steps ? softplus_fast(z) : 0.f;  // delta = 0 past the end: h unchanged
+      du[i] = dl[i] * uv;
+      Du[i] = Dv * uv;
     }
-    __syncthreads();
-    // ---- phase B: the recurrence, TC steps
-    for (int t = 0; t < tc; ++t) {
-      const float dlt = dt_s[t * CE + c];
-      const float uv = u_s[t * CE + c];
-      const float du = dlt * uv;
-      float yp = 0.f;
+    // ---- delta and delta*u of all 16 steps of the chunk, in every lane
+    float dls[kScanChunk], dus[kScanChunk];
 #pragma unroll
-      for (int j = 0; j < NPT; ++j) {
-        const int n = g * NPT + j;
-        const float a = ex2_approx(dlt * A2[j]);
-        h[j] = fmaf(a, h[j], du * B_s[t * kScanN + n]);
-        yp = fmaf(C_s[t * kScanN + n], h[j], yp);
+    for (int tl = 0; tl < kScanChunk; ++tl) {
+      const int i = tl / TPC, s2 = tl % TPC;
+      dls[tl] = TPC > 1 ? __shfl_sync(0xffffffffu, dl[i], src0 + s2) : dl[i];
+      dus[tl] = TPC > 1 ? __shfl_sync(0xffffffffu, du[i], src0 + s2) : du[i];
+    }
+    // ---- advance the states through the chunk.  The decay factors of step
+    // tl+1 are issued before the state updates of step tl, so each exp2 has
+    // a full step of independent work between it and its use.
+    float ys[SPL];
+    float a_cur[NPT];
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) a_cur[j] = ex2_approx(dls[0] * A2[j]);
+    float yp[TPC];
+#pragma unroll
+    for (int tl = 0; tl < kScanChunk; ++tl) {
+      float a_nxt[NPT];
+      if (tl + 1 < kScanChunk) {
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) a_nxt[j] = ex2_approx(dls[tl + 1] * A2[j]);
       }
+      const float4* Bp = reinterpret_cast<const float4*>(B_s + tl * kScanN + g * NPT);
+      const float4* Cp = reinterpret_cast<const float4*>(C_s + tl * kScanN + g * NPT);
+      const float du_s = dus[tl];
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int o = TPC / 2; o > 0; o >>= 1) yp += __shfl_xor_sync(0xffffffffu, yp, o);
-      if (g == 0) y_s[t * CE + c] = fmaf(Dv, uv, yp);
+      for (int v = 0; v < NPT / 4; ++v) {
+        const float4 b4 = Bp[v];
+        const float4 c4 = Cp[v];
+        h[4 * v + 0] = fmaf(a_cur[4 * v + 0], h[4 * v + 0], du_s * b4.x);
+        h[4 * v + 1] = fmaf(a_cur[4 * v + 1], h[4 * v + 1], du_s * b4.y);
+        h[4 * v + 2] = fmaf(a_cur[4 * v + 2], h[4 * v + 2], du_s * b4.z);
+        h[4 * v + 3] = fmaf(a_cur[4 * v + 3], h[4 * v + 3], du_s * b4.w);
+        acc0 = fmaf(c4.x, h[4 * v + 0], acc0);
+        acc1 = fmaf(c4.y, h[4 * v + 1], acc1);
+        acc0 = fmaf(c4.z, h[4 * v + 2], acc0);
+        acc1 = fmaf(c4.w, h[4 * v + 3], acc1);
+      }
+      yp[tl % TPC] = acc0 + acc1;
+      if (tl % TPC == TPC - 1) ys[tl / TPC] = reduce_scatter<TPC>(yp, g) + Du[tl / TPC];
+      if (tl + 1 < kScanChunk) {
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) a_cur[j] = a_nxt[j];
+      }
     }
-    __syncthreads();
-    // ---- phase C: write the chunk's outputs
-    for (int i = tid; i < kScanTC * CE; i += 128) {
-      const int t = i / CE, cc = i - t * CE;
-      if (t < tc && e0 + cc < E)
-        store_as(reinterpret_cast<Ty*>(P.y) + (tok0 + t0 + t) * E + e0 + cc, y_s[i]);
+    if (ch_ok) {
+#pragma unroll
+      for (int i = 0; i < SPL; ++i) {
+        const int tl = i * TPC + g;
+        if (tl < steps) store_as(yrow + (long)(t0 + tl) * E, ys[i]);
+      }
     }
   }
   if (P.h_last != nullptr && ch_ok) {

@@ -52,6 +52,26 @@ __device__ __forceinline__ int quant_code(float v, float sigma) {
   return max(-128, min(127, q));
 }
 
+// Exact conversions on the FMA/ALU pipes for |x| < 2^22, through the float
+// 1.5 * 2^23 (bit pattern 0x4B400000), whose ulp is 1: adding an integer-
+// valued or real x lands in [2^23, 2^24), where the IEEE round-to-nearest-
+// even addition performs rint(x) and the low mantissa bits hold rint(x) in
+// two's complement.
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
+__device__ __forceinline__ float i2f_exact(int a) { return __int_as_float(a + kMagicBits) - kMagic; }
+// Bit pattern whose low byte is the int8 code rint(v * sigma).  With
+// sigma = 127 / max|v| the product never exceeds 127 in magnitude (so the
+// clamp to [-128, 127] of the definition never binds).  Both steps are
+// IEEE round-to-nearest (no contraction into an FMA).
+__device__ __forceinline__ uint32_t code_bits(float v, float sigma) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, sigma), kMagic));
+}
+// Four codes (low bytes of four code_bits words) packed into one word.
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 // One warp per row.  x [M, K] (row pitch ldx elements) -> q int8 [M, ldq]
 // (columns K..ldq-1 written as 0), deq [M].  The row is read twice (the
 // second time from L1/L2): once for max|v| and sum(v^2), once for the codes.
@@ -86,6 +106,76 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ x
       }
       *reinterpret_cast<uint32_t*>(qr + k0) = word;
     }
+    if (lane == 0) {
+      const float r = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
+      deq[row] = mx * r / 127.f;
+    }
+  }
+}
+
+// Vector form of quant_rows_kernel for rows of at most VPL*32 16-byte
+// vectors: every lane loads its vectors once into registers (16-byte loads,
+// coalesced across the warp), and writes its codes as one 4- or 8-byte store
+// per vector.  Requires K and ldx multiples of the vector width and a
+// 16-byte aligned x.
+template <typename T, int VPL>
+__global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict__ x, int M, int K,
+                                                             long ldx, int8_t* __restrict__ q,
+                                                             long ldq, float* __restrict__ deq) {
+  constexpr int EPV = 16 / (int)sizeof(T);  // elements per vector
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const T* xr = x + row * ldx;
+    float v[VPL][EPV];
+    float mx = 0.f, ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int k0 = (i * 32 + lane) * EPV;
+      if (k0 < K) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xr + k0));
+        if constexpr (sizeof(T) == 4) {
+          v[i][0] = __uint_as_float(raw.x);
+          v[i][1] = __uint_as_float(raw.y);
+          v[i][2] = __uint_as_float(raw.z);
+          v[i][3] = __uint_as_float(raw.w);
+        } else {
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[i][2 * j] = __uint_as_float(w[j] << 16);
+            v[i][2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) v[i][j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < EPV; ++j) {
+        mx = fmaxf(mx, fabsf(v[i][j]));
+        ss = fmaf(v[i][j], v[i][j], ss);
+      }
+    }
+    mx = warp_max(mx);
+    ss = warp_sum(ss);
+    const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+    int8_t* qr = q + row * ldq;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int k0 = (i * 32 + lane) * EPV;
+      if (k0 < K) {
+        uint32_t w[EPV / 4];
+#pragma unroll
+        for (int j4 = 0; j4 < EPV / 4; ++j4)
+          w[j4] = pack4(code_bits(v[i][4 * j4], sigma), code_bits(v[i][4 * j4 + 1], sigma),
+                        code_bits(v[i][4 * j4 + 2], sigma), code_bits(v[i][4 * j4 + 3], sigma));
+        if constexpr (EPV == 4) *reinterpret_cast<uint32_t*>(qr + k0) = w[0];
+        else *reinterpret_cast<uint2*>(qr + k0) = make_uint2(w[0], w[1]);
+      }
+    }
+    for (int k = K + lane; k < ldq; k += 32) qr[k] = 0;
     if (lane == 0) {
       const float r = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
       deq[row] = mx * r / 127.f;
@@ -229,6 +319,8 @@ struct ExpandJob {
   int row0;
   void* dst;
   int ld;
+  float* s_t;   // bf16 expansion: transposed group scales [G][ld_s] (rows row0..)
+  long ld_s;
 };
 struct ExpandJobs {
   ExpandJob job[8];
@@ -259,39 +351,49 @@ __device__ __forceinline__ uint4 expand16_i8(uint32_t p) {
   return o;
 }
 
-// int8 expansion: each thread writes 16 consecutive elements of one row.
-__global__ void __launch_bounds__(256) expand_i8_kernel(ExpandJobs jobs) {
-  for (int ji = 0; ji < jobs.count; ++ji) {
-    const ExpandJob J = jobs.job[ji];
-    const int kb = (J.k_in + 3) / 4;
+// int8 expansion over one flat index space covering every job: each thread
+// writes 16 consecutive elements (one 32-bit word of packed codes) of one
+// row.  `first[j]` is the first flat index of job j (first[count] = total).
+__global__ void __launch_bounds__(256) expand_i8_kernel(ExpandJobs jobs, int4 first_lo,
+                                                        int4 first_hi) {
+  const int first[8] = {first_lo.x, first_lo.y, first_lo.z, first_lo.w,
+                        first_hi.x, first_hi.y, first_hi.z, first_hi.w};
+  const int total = first[jobs.count];
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    int ji = 0;
+#pragma unroll
+    for (int k = 1; k < 7; ++k)
+      if (k < jobs.count && i >= first[k]) ji = k;
+    const ExpandJob& J = jobs.job[ji];
     const int chunks = J.ld / 16;
-    const long total = (long)J.n_out * chunks;
-    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (long)gridDim.x * blockDim.x) {
-      const long n = i / chunks;
-      const int ch = (int)(i - n * chunks);
-      const uint8_t* src = J.packed + n * kb;
-      uint32_t p = 0x55555555u;  // code 1 (w = 0) in every slot
+    const int li = i - first[ji];
+    const int n = li / chunks;
+    const int ch = li - n * chunks;
+    const int kb = (J.k_in + 3) / 4;
+    const uint8_t* src = J.packed + (long)n * kb;
+    uint32_t p;
+    if ((kb & 3) == 0 && ch * 4 + 4 <= kb) {
+      p = __ldg(reinterpret_cast<const uint32_t*>(src) + ch);
+    } else {
+      p = 0x55555555u;  // code 1 (w = 0) in every slot
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         const int byte = ch * 4 + b;
-        const uint32_t v = byte < kb ? src[byte] : 0x55u;
-        p = (p & ~(0xffu << (8 * b))) | (v << (8 * b));
+        if (byte < kb) p = (p & ~(0xffu << (8 * b))) | ((uint32_t)src[byte] << (8 * b));
       }
-      uint4 o = expand16_i8(p);
-      // zero columns >= k_in (padding codes inside the last byte already are 0)
-      int8_t* dst = reinterpret_cast<int8_t*>(J.dst) + (long)(J.row0 + n) * J.ld + ch * 16;
-      *reinterpret_cast<uint4*>(dst) = o;
     }
+    *reinterpret_cast<uint4*>(reinterpret_cast<int8_t*>(J.dst) + (long)(J.row0 + n) * J.ld + ch * 16) =
+        expand16_i8(p);
   }
 }
 
-// bf16 expansion with the group scale folded in: element = w * bf16(s[n, k/group]).
+// bf16 expansion: exact ternary values {-1, 0, 1} (the group scales are
+// applied in fp32 by the GEMM epilogue), 8 elements per thread, plus the
+// transposed fp32 group scales s_t[g][row0 + n] = s[n, g] (s[0] for group 0).
 __global__ void __launch_bounds__(256) expand_bf16_kernel(ExpandJobs jobs) {
   for (int ji = 0; ji < jobs.count; ++ji) {
     const ExpandJob J = jobs.job[ji];
     const int kb = (J.k_in + 3) / 4;
-    const int ng = J.group > 0 ? (J.k_in + J.group - 1) / J.group : 1;
     const int chunks = J.ld / 8;
     const long total = (long)J.n_out * chunks;
     for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -309,9 +411,8 @@ __global__ void __launch_bounds__(256) expand_bf16_kernel(ExpandJobs jobs) {
           uint32_t bits = 0;
           if (k < J.k_in) {
             const int c = (src[k >> 2] >> (2 * (k & 3))) & 3;
-            const float s = J.group > 0 ? J.scales[n * ng + k / J.group] : J.scales[0];
-            const float w = (float)(c - 1) * __bfloat162float(__float2bfloat16_rn(s));
-            bits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(w));
+            // bf16 bit patterns of -1, 0, +1
+            bits = c == 0 ? 0xBF80u : (c == 2 ? 0x3F80u : 0u);
           }
           pair |= bits << (16 * h);
         }
@@ -319,6 +420,17 @@ __global__ void __launch_bounds__(256) expand_bf16_kernel(ExpandJobs jobs) {
       }
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(J.dst) + (long)(J.row0 + n) * J.ld + ch * 8;
       *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (J.s_t != nullptr) {
+      const int G = (J.k_in + 127) / 128;
+      const int ng = J.group > 0 ? (J.k_in + J.group - 1) / J.group : 1;
+      const long nsc = (long)G * J.n_out;
+      for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < nsc;
+           i += (long)gridDim.x * blockDim.x) {
+        const int g = (int)(i / J.n_out);
+        const int n = (int)(i - (long)g * J.n_out);
+        J.s_t[(long)g * J.ld_s + J.row0 + n] = J.group > 0 ? J.scales[(long)n * ng + g] : J.scales[0];
+      }
     }
   }
 }

@@ -55,7 +55,7 @@ class DeviceLayer:
         self.layer = abi.bitssm_layer(
             m["W_in"].tw, m["W_dt_down"].tw, m["W_B"].tw, m["W_C"].tw, m["W_dt_up"].tw,
             m["W_out"].tw, self.A.data_ptr(), self.D.data_ptr(), self.dt_bias.data_ptr(),
-            lw.W_in.shape[1], lw.W_in.shape[0], lw.A.shape[1], lw.W_dt_down.shape[0], None)
+            lw.W_in.shape[1], lw.W_in.shape[0], lw.A.shape[1], lw.W_dt_down.shape[0], None, 0)
         self._prepared = None
 
     def prepare(self, stream=None):

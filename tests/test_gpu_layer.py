@@ -27,10 +27,12 @@ def env(cuda_ok):
     return torch, abi, dev
 
 
-def run_layers(env, x, layers, act, dtype, prepare=False, residual=False):
+def run_layers(env, x, layers, act, dtype, prepare=False, residual=False, keep_codes=True):
     torch, abi, dev = env
     B, L, d = x.shape
     dl = [dev.DeviceLayer(lw, act) for lw in layers]
+    for dd in dl:
+        dd.layer.flags = abi.KEEP_CODES if keep_codes else 0
     if prepare:
         for dd in dl:
             dd.prepare()
@@ -121,11 +123,38 @@ def test_trissm_bf16_layer_stages(env):
 
 @pytest.mark.parametrize("B,L", [(1, 1), (3, 37), (2, 129), (5, 64)])
 def test_ragged_shapes_a8(env, B, L):
+    # d_model = 64: the six-kernel path
     torch, abi, dev = env
     wl = S.WORKLOADS["tiny"]
     x, layers = S.make_inputs(wl, seed=B * 100 + L, batch=B, seqlen=L)
     out, ws, dl = run_layers(env, x, layers, abi.A8, abi.F32)
     a8_stage_checks(env, x, layers[0], ws, dl[0], out, abi.F32)
+
+
+@pytest.mark.parametrize("B,L,dt", [(1, 1, "f32"), (3, 37, "bf16"), (2, 129, "f32"), (1, 300, "bf16")])
+def test_ragged_shapes_a8_fused(env, B, L, dt):
+    # d_model = 256, d_inner = 512: the fused pre / scan / post path, with
+    # token counts that leave a partial 128-token tile
+    torch, abi, dev = env
+    wl = S.WORKLOADS["trissm"]
+    x, layers = S.make_inputs(wl, seed=B * 10 + L, batch=B, seqlen=L)
+    dtype = abi.F32 if dt == "f32" else abi.BF16
+    if dt == "f32":
+        x = S.random_rows(B + L, B * L, 256).reshape(B, L, 256)
+    out, ws, dl = run_layers(env, x, layers, abi.A8, dtype)
+    assert abi.bitssm_forward_launches(dl[0].layer, abi.A8) == 4
+    a8_stage_checks(env, x, layers[0], ws, dl[0], out, dtype)
+
+
+def test_fused_codes_flag_does_not_change_results(env):
+    torch, abi, dev = env
+    wl = S.WORKLOADS["trissm"]
+    x, layers = S.make_inputs(wl, seed=4, batch=4)
+    o1, _, _ = run_layers(env, x, layers, abi.A8, abi.BF16, keep_codes=True)
+    o2, ws, dl = run_layers(env, x, layers, abi.A8, abi.BF16, keep_codes=False)
+    assert np.array_equal(o1, o2)
+    v = abi.bitssm_workspace_layout(dl[0].layer, 4, 256, abi.BF16, abi.A8)
+    assert v.q_x == v.q_u == v.q_y == 2 ** 64 - 1
 
 
 def test_prepared_weights_residual_and_determinism(env):
@@ -184,7 +213,7 @@ def test_stack12_teacher_forced_per_layer(env):
     ref_stack, _ = O.bitssm_stack(x, [O.TernaryLayer(lw, "A8") for lw in layers])
     diff = out.astype(np.float64) - ref_stack
     assert norm_err(out, ref_stack) <= TOL_BF16
-    assert np.sqrt((diff ** 2).mean() / (ref_stack ** 2).mean()) <= 5e-3
+    assert np.sqrt((diff ** 2).mean() / (ref_stack ** 2).mean()) <= TOL_BF16
     print(f"stack12 end to end: max elementwise {rel_err(out, ref_stack):.3e}, "
           f"normwise {norm_err(out, ref_stack):.3e}")
 

@@ -41,9 +41,10 @@ def oracle_scan(u, dr, bias, A, Bm, Cm, D, h0=None):
     return O.selective_scan(u, delta, A, Bm, Cm, D, h0)
 
 
-# (B, L, E): covers NPT = 16 (many channels), 4 and 1, ragged L and E
+# (B, L, E): covers 16, 8 and 4 states per thread (many to few channels),
+# ragged L and E
 SHAPES = [(1, 64, 128), (2, 37, 40), (3, 1, 16), (64, 256, 512), (1, 300, 8), (4, 2048, 96),
-          (16, 33, 4096), (32, 20, 4096)]
+          (16, 33, 4096), (32, 20, 4096), (4, 70, 4096)]
 
 
 @pytest.mark.parametrize("B,L,E", SHAPES)
