@@ -157,13 +157,10 @@ def run_ours(args):
     T = B * L
     x, layers = S.make_inputs(wl, seed=rank)
     dl = [dev.DeviceLayer(lw, act) for lw in layers]
-    stream = torch.cuda.current_stream()
     xd = dev.to_device_input(x, dtype)
     out = torch.empty_like(xd)
-    nbytes = abi.bitssm_workspace_size(dl[0].layer, B, L, dtype, act)
-    ws = dev.Workspace(nbytes)
-    nl = abi.bitssm_forward_launches(dl[0].layer, act)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    n_layers = len(dl)
 
     def new_events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -171,82 +168,103 @@ def run_ours(args):
             e.record()  # creates the underlying cudaEvent_t
         return evs
 
-    n_layers = len(dl)
-    per_step = n_layers * (nl + 1)
+    def timed(prepared: bool, sample_clocks: bool):
+        """K forwards (CUDA-graph replays); returns per-step ms and per-kernel ms."""
+        for d_l in dl:
+            if prepared:
+                d_l.prepare()
+            else:
+                d_l.unprepare()
+        nbytes = abi.bitssm_workspace_size(dl[0].layer, B, L, dtype, act)
+        ws = dev.Workspace(nbytes)
+        nl = abi.bitssm_forward_launches(dl[0].layer, act)
+        per_step = n_layers * (nl + 1)
 
-    def step(evs):
-        """One forward; evs: (nl + 1) events per layer, recorded by the library
-        before every kernel and after the last."""
-        st = torch.cuda.current_stream()
-        h_in = xd
-        for li, d_l in enumerate(dl):
-            e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
-            abi.bitssm_forward_timed(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B, L,
-                                     dtype, act, ws.addr, nbytes, [ev.cuda_event for ev in e], st)
-            h_in = out
-
-    # eager warm-up (also sets the kernels' shared-memory attributes)
-    warm = new_events(per_step)
-    for _ in range(args.warmup):
-        flush.zero_()
-        step(warm)
-    torch.cuda.synchronize()
-
-    # The timed steps run as CUDA-graph replays (host launch cost out of the
-    # device timeline): one graph holds G x (L2 flush + timed forward).
-    G = max(1, min(args.steps, 100))
-    R = (args.steps + G - 1) // G
-    K = G * R
-    gevents = [new_events(per_step) for _ in range(G)]
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.graph(graph, stream=cap):
-        for i in range(G):
-            flush.zero_()
-            step(gevents[i])
-    torch.cuda.synchronize()
-    graph.replay()  # one untimed replay
-    torch.cuda.synchronize()
-
-    props = torch.cuda.get_device_properties(local)
-    gpu_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
-    sampler = ClockSampler(gpu_id)
-    if rank == 0:
-        sampler.start()
-        time.sleep(0.3)
-    step_ms, kern_ms = [], [[0.0] * nl for _ in range(n_layers)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_wall = time.perf_counter()
-    for r in range(R):
-        graph.replay()
-        torch.cuda.synchronize()
-        for evs in gevents:
-            tot = 0.0
-            for li in range(n_layers):
+        def step(evs):
+            """One forward; evs: (nl + 1) events per layer, recorded by the
+            library before every kernel and after the last."""
+            st = torch.cuda.current_stream()
+            h_in = xd
+            for li, d_l in enumerate(dl):
                 e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
-                for i in range(nl):
-                    kern_ms[li][i] += e[i].elapsed_time(e[i + 1])
-                tot += e[0].elapsed_time(e[nl])
-            step_ms.append(tot)
-    torch.cuda.synchronize()
-    t_wall = time.perf_counter() - t_wall
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if rank == 0 else None
-    del graph
-    args.steps = K
+                abi.bitssm_forward_timed(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B,
+                                         L, dtype, act, ws.addr, nbytes,
+                                         [ev.cuda_event for ev in e], st)
+                h_in = out
 
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
+        # eager warm-up (also sets the kernels' shared-memory attributes)
+        warm = new_events(per_step)
+        for _ in range(args.warmup):
+            flush.zero_()
+            step(warm)
+        torch.cuda.synchronize()
+        # The timed steps run as CUDA-graph replays (host launch cost out of
+        # the device timeline): one graph holds G x (L2 flush + forward).
+        G = max(1, min(args.steps, 100))
+        R = (args.steps + G - 1) // G
+        gevents = [new_events(per_step) for _ in range(G)]
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(graph, stream=cap):
+            for i in range(G):
+                flush.zero_()
+                step(gevents[i])
+        torch.cuda.synchronize()
+        graph.replay()  # one untimed replay
+        torch.cuda.synchronize()
+        sampler = None
+        if sample_clocks and rank == 0:
+            props = torch.cuda.get_device_properties(local)
+            gpu_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            sampler = ClockSampler(gpu_id)
+            sampler.start()
+            time.sleep(0.3)
+        step_ms, kern_ms = [], [[0.0] * nl for _ in range(n_layers)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter()
+        for _ in range(R):
+            graph.replay()
+            torch.cuda.synchronize()
+            for evs in gevents:
+                tot = 0.0
+                for li in range(n_layers):
+                    e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
+                    for i in range(nl):
+                        kern_ms[li][i] += e[i].elapsed_time(e[i + 1])
+                    tot += e[0].elapsed_time(e[nl])
+                step_ms.append(tot)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+        if world > 1:
+            dist.barrier()
+        clocks = sampler.stop() if sampler is not None else None
+        del graph
+        total_ms = sum(step_ms)
+        if world > 1:
+            t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            total_ms = float(t.item())
+        K = G * R
+        return dict(ms=total_ms / K, kern_ms=kern_ms, nl=nl, K=K, G=G, R=R, t_wall=t_wall,
+                    clocks=clocks, ws=ws, nbytes=nbytes)
+
+    # the hot path: weights expanded once (bitssm_prepare_weights), then every
+    # forward of the timed region runs every stage on fresh activations
+    main = timed(prepared=True, sample_clocks=True)
+    # the same forward when the packed weights are expanded inside every call
+    unprep = timed(prepared=False, sample_clocks=False)
+    for d_l in dl:
+        d_l.prepare()
+    nl, kern_ms, clocks, t_wall = main["nl"], main["kern_ms"], main["clocks"], main["t_wall"]
+    ws, nbytes = main["ws"], main["nbytes"]
+    args.steps = main["K"]
+    ms_per_step = main["ms"]
     value = T * world / (ms_per_step / 1e3)
+    G, R = main["G"], main["R"]
 
     # ---------------- end to end through the C ABI with host buffers
     x_host = torch.empty(xd.shape, dtype=xd.dtype, pin_memory=True)
@@ -292,7 +310,7 @@ def run_ours(args):
         return
 
     # ---------------- roofline of the dominant kernel
-    if act == abi.A8 and nl in (3, 4):
+    if act == abi.A8 and nl == 3:
         names = ["expand_weights", "bitssm_pre(quant_x+in_proj+x_proj)",
                  "selective_scan_fused_dt", "bitssm_post(quant_y+out_proj)"]
     elif act == abi.A8:
@@ -347,6 +365,8 @@ def run_ours(args):
         "roofline": roof,
         "kernel_share": share,
         "kernel_avg_us": {names[i]: round(avg_kernel_ms[i] * 1e3, 2) for i in range(nl)},
+        "weights": "expanded once before the timed region (bitssm_prepare_weights)",
+        "value_with_per_call_weight_expansion": round(T * world / (unprep["ms"] / 1e3), 1),
         "layer_hbm_gbs_algorithmic": round(layer_gbs, 1),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes},

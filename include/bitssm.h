@@ -53,7 +53,7 @@ enum bitssm_status_code {
   BITSSM_ERR_DEVICE_FLAG = 6       /* another device-side check failed */
 };
 
-enum bitssm_dtype { BITSSM_F32 = 0, BITSSM_BF16 = 1, BITSSM_I32 = 2 };
+enum bitssm_dtype { BITSSM_F32 = 0, BITSSM_BF16 = 1, BITSSM_I32 = 2, BITSSM_I16 = 3 };
 
 /* Activation modes.  A8: per-token absmax int8 activation codes (BitNet
  * b1.58; TriSSM README opening paragraph).  A16: bf16 activations without
@@ -246,7 +246,9 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
  * (size_t)-1 for a buffer the forward does not write (the A8 codes q_x,
  * q_u and q_y are written only with BITSSM_KEEP_CODES when the layer runs
  * as the fused kernels), and the row pitch in elements of each buffer.
- *   A8:  q_x int8 [T, ld_qx], deq_x float [T], u float [T, E],
+ *   A8:  q_x int8 [T, ld_qx], deq_x float [T], u [T, E] of u_dtype (float,
+ *        or, in the fused kernels, the exact int16 in_proj accumulators with
+ *        u = u_i16 * u_scale[t], u_scale float [T]),
  *        q_u int8 [T, ld_qu], deq_u float [T], Bm float [T, N],
  *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],
  *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]
@@ -258,7 +260,9 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
 typedef struct bitssm_ws_view {
   size_t q_x, deq_x, u, q_u, deq_u, Bm, Cm, q_dt, deq_dt, y, q_y, deq_y;
   size_t r_x, dt_low, r_dt, delta_raw, r_y;
+  size_t u_scale;
   int ld_qx, ld_qu, ld_qdt;
+  int u_dtype;
 } bitssm_ws_view;
 int bitssm_workspace_layout(const bitssm_layer* p, int B, int L, int dtype, int act_mode,
                             bitssm_ws_view* view);

@@ -26,7 +26,7 @@ ERR_CUDA = 4
 ERR_TIMEOUT = 5
 ERR_DEVICE_FLAG = 6
 
-F32, BF16, I32 = 0, 1, 2
+F32, BF16, I32, I16 = 0, 1, 2, 3
 A8, A16 = 0, 1
 KEEP_CODES = 1
 
@@ -69,8 +69,8 @@ class bitssm_layer(ctypes.Structure):
 class bitssm_ws_view(ctypes.Structure):
     _fields_ = [(n, _sz) for n in ("q_x", "deq_x", "u", "q_u", "deq_u", "Bm", "Cm", "q_dt",
                                    "deq_dt", "y", "q_y", "deq_y", "r_x", "dt_low", "r_dt",
-                                   "delta_raw", "r_y")] + \
-               [("ld_qx", _i), ("ld_qu", _i), ("ld_qdt", _i)]
+                                   "delta_raw", "r_y", "u_scale")] + \
+               [("ld_qx", _i), ("ld_qu", _i), ("ld_qdt", _i), ("u_dtype", _i)]
 
 
 _P_TW = ctypes.POINTER(bitssm_tw)

@@ -273,6 +273,7 @@ int launch_scan_rv(const ScanParams& P, cudaStream_t st) {
 
 template <bool FUSED, typename Tu, typename Td, typename Ty>
 int launch_scan(const ScanParams& P, cudaStream_t st) {
+  if (std::is_same<Tu, int16_t>::value != (P.u_scale != nullptr)) return BITSSM_ERR_INVALID_ARG;
   if constexpr (FUSED) {
     switch (P.R / 16) {  // Delta-up width (dt_rank padded to 16)
       case 1: return launch_scan_rv<true, 1, Tu, Td, Ty>(P, st);
@@ -374,6 +375,8 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   bitssm_ws_view& v = P.v;
   v.q_x = v.deq_x = v.u = v.q_u = v.deq_u = v.Bm = v.Cm = v.q_dt = v.deq_dt = v.y = v.q_y = v.deq_y = none;
   v.r_x = v.dt_low = v.r_dt = v.delta_raw = v.r_y = none;
+  v.u_scale = none;
+  v.u_dtype = P.a16 ? BITSSM_BF16 : BITSSM_F32;
   P.ss_u = none;
   auto take = [&](size_t bytes) {
     size_t r = a;
@@ -387,6 +390,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
     v.q_x = take(T * P.ld_d);
     v.deq_x = take(T * 4);
     v.u = take(T * P.E * 4);
+    v.u_scale = take(T * 4);
     v.q_u = take(T * P.ld_E);
     v.deq_u = take(T * 4);
     v.Bm = take(T * P.N * 4);
@@ -486,7 +490,7 @@ T* at(void* base, size_t off) {
 // Whether the A8 layer runs as the fused pre kernel + scan + post kernel:
 // d_model of 128 or 256, d_inner of 256 or 512, dt_rank + 2 d_state <= 64.
 bool a8_fused(const LayerPlan& P) {
-  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64;
+  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64 && P.R <= 64;
 }
 
 template <typename Tx, int BN1, int K1P>
@@ -557,7 +561,8 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
     Q.x = x; Q.M = P.T; Q.d = P.d; Q.E = P.E; Q.xrows = P.xrows; Q.R = P.R; Q.Ns = P.N;
     Q.s_in = p->in_proj.scales; Q.s_dt = p->dt_down.scales; Q.s_B = p->b_proj.scales;
     Q.s_C = p->c_proj.scales;
-    Q.u = at<float>(ws, v.u); Q.deq_x = at<float>(ws, v.deq_x); Q.deq_u = at<float>(ws, v.deq_u);
+    Q.u = at<int16_t>(ws, v.u); Q.u_scale = at<float>(ws, v.u_scale);
+    Q.deq_x = at<float>(ws, v.deq_x); Q.deq_u = at<float>(ws, v.deq_u);
     Q.q_dt = at<int8_t>(ws, v.q_dt); Q.ld_qdt = P.ld_R; Q.deq_dt = at<float>(ws, v.deq_dt);
     Q.Bm = at<float>(ws, v.Bm); Q.Cm = at<float>(ws, v.Cm);
     if (keep) {
@@ -573,7 +578,7 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
   {
     ScanParams S;
     std::memset(&S, 0, sizeof(S));
-    S.u = at<float>(ws, v.u);
+    S.u = at<int16_t>(ws, v.u); S.u_scale = at<float>(ws, v.u_scale);
     S.q_dt = at<int8_t>(ws, v.q_dt); S.ld_qdt = P.ld_R;
     S.deq_dt = at<float>(ws, v.deq_dt);
     S.W_up = reinterpret_cast<const int8_t*>(wexp + P.w_up); S.ld_w = P.ld_R;
@@ -583,7 +588,7 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
     S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
     S.y = at<float>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
-    rc = launch_scan<true, float, float, float>(S, st);
+    rc = launch_scan<true, int16_t, float, float>(S, st);
     if (rc) return rc;
   }
   mk.mark();
@@ -996,8 +1001,12 @@ int bitssm_workspace_layout(const bitssm_layer* p, int B, int L, int dtype, int 
   if (rc) return rc;
   const LayerPlan P = plan_layer(p, B, L, act_mode, p->prepared != nullptr);
   *view = P.v;
-  if (act_mode == BITSSM_A8 && a8_fused(P) && !(p->flags & BITSSM_KEEP_CODES))
-    view->q_x = view->q_u = view->q_y = (size_t)-1;
+  if (act_mode == BITSSM_A8 && a8_fused(P)) {
+    view->u_dtype = BITSSM_I16;
+    if (!(p->flags & BITSSM_KEEP_CODES)) view->q_x = view->q_u = view->q_y = (size_t)-1;
+  } else {
+    view->u_scale = (size_t)-1;
+  }
   return BITSSM_OK;
 }
 

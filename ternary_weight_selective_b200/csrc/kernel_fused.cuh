@@ -116,6 +116,33 @@ __device__ __forceinline__ void warp_store_block(float* sbuf, const float (&v)[3
   __syncwarp();
 }
 
+// One warp stores a 32-row x 32-column block of int16 values, row i held
+// by lane i as 16 words of two int16 each, through its shared buffer: rows
+// of 64 bytes whose four 16-byte chunks are permuted by (row / 2) % 4 so
+// that neither the row writes nor the read-back hit a bank twice; each
+// store instruction covers 8 rows of 64 contiguous bytes.  Rows >= M are
+// skipped.
+__device__ __forceinline__ void warp_store_block_i16(uint32_t* sbuf, const uint32_t (&w)[16], int lane,
+                                                     int16_t* out, long ld, long row0, int col0,
+                                                     long M) {
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    *reinterpret_cast<uint4*>(sbuf + lane * 16 + ((k ^ sw) << 2)) =
+        make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int r = it * 8 + (lane >> 2);
+    const int k = lane & 3;  // 16-byte chunk of the row
+    const long m = row0 + r;
+    if (m < M)
+      *reinterpret_cast<uint4*>(out + m * ld + col0 + 8 * k) =
+          *reinterpret_cast<const uint4*>(sbuf + r * 16 + ((k ^ ((r >> 1) & 3)) << 2));
+  }
+  __syncwarp();
+}
+
 // Load EPL consecutive elements (EPL * sizeof(T) a multiple of 8 bytes, the
 // address aligned to it) as floats.
 template <typename T, int EPL>
@@ -182,12 +209,28 @@ __device__ __forceinline__ void quantize_rows_to_smem(const T* __restrict__ x, l
       mx = warp_max(mx);
       ss = warp_sum(ss);
       const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+      // this lane's EPL codes are contiguous in one 16-byte chunk of the row
+      uint32_t w[EPL / 4];
 #pragma unroll
-      for (int j0 = 0; j0 < EPL; j0 += 4) {
-        const uint32_t w = pack4(code_bits(v[b][j0], sigma), code_bits(v[b][j0 + 1], sigma),
-                                 code_bits(v[b][j0 + 2], sigma), code_bits(v[b][j0 + 3], sigma));
-        *reinterpret_cast<uint32_t*>(a_s + sw128_off(row, lane * EPL + j0)) = w;
-        if (q_g != nullptr && m < M) *reinterpret_cast<uint32_t*>(q_g + m * ldq + lane * EPL + j0) = w;
+      for (int j0 = 0; j0 < EPL; j0 += 4)
+        w[j0 / 4] = pack4(code_bits(v[b][j0], sigma), code_bits(v[b][j0 + 1], sigma),
+                          code_bits(v[b][j0 + 2], sigma), code_bits(v[b][j0 + 3], sigma));
+#pragma unroll
+      for (int c0 = 0; c0 < EPL; c0 += 16) {
+        const int k = lane * EPL + c0;
+        uint8_t* dst = a_s + sw128_off(row, k);
+        int8_t* gdst = (q_g != nullptr && m < M) ? q_g + m * ldq + k : nullptr;
+        if constexpr (EPL >= 16) {
+          const uint4 q4 = make_uint4(w[c0 / 4], w[c0 / 4 + 1], w[c0 / 4 + 2], w[c0 / 4 + 3]);
+          *reinterpret_cast<uint4*>(dst) = q4;
+          if (gdst) *reinterpret_cast<uint4*>(gdst) = q4;
+        } else if constexpr (EPL == 8) {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+          if (gdst) *reinterpret_cast<uint2*>(gdst) = make_uint2(w[0], w[1]);
+        } else {
+          *reinterpret_cast<uint32_t*>(dst) = w[0];
+          if (gdst) *reinterpret_cast<uint32_t*>(gdst) = w[0];
+        }
       }
       if (lane == 0) {
         const float r = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
@@ -208,7 +251,8 @@ struct PreParams {
   const float* s_dt;
   const float* s_B;
   const float* s_C;
-  float* u;             // [M, E] f32
+  int16_t* u;           // [M, E] int16: the exact in_proj accumulators (|acc| <= 127 d)
+  float* u_scale;       // [M]: u = u * u_scale (s_in * deq_x)
   float* deq_x;         // [M] (inspection)
   float* deq_u;         // [M] (inspection)
   int8_t* q_dt;         // [M, ld_qdt]
@@ -224,8 +268,9 @@ struct PreParams {
 
 // Shared-memory plan of the pre kernel (bytes, 1024-aligned regions):
 //   phase 1: A1 codes of x [K1P panels x 16 KB] | W_in [K1P panels x BN1*128]
-//   phase 2: A2 codes of u [E/128 panels x 16 KB] | u transpose buffers |
-//            W_x [E/128 panels x BN2*128]  (reusing phase 1's space)
+//   phase 2: A2 codes of u [E/128 panels x 16 KB] | u transpose buffers
+//            (reusing phase 1's space once the in_proj MMAs are done)
+//   always:  W_x [E/128 panels x BN2*128] after phase 1, loaded at start
 template <int BN1, int K1P, int BN2>
 struct PreCfg {
   static constexpr int kA1 = K1P * 16384;
@@ -234,10 +279,10 @@ struct PreCfg {
   static constexpr int kE1P = BN1 / 128;  // x_proj K panels (E <= BN1)
   static constexpr int kA2 = kE1P * 16384;
   static constexpr int kStg = kFusedWorkers * kStageFloats * 4;
-  static constexpr int kW2Off = ((kA2 + kStg) + 1023) / 1024 * 1024;
+  static constexpr int kPhase2 = kA2 + kStg;
+  static constexpr int kW2Off = ((kPhase1 > kPhase2 ? kPhase1 : kPhase2) + 1023) / 1024 * 1024;
   static constexpr int kW2 = kE1P * BN2 * 128;
-  static constexpr int kPhase2 = kW2Off + kW2;
-  static constexpr int kMain = kPhase1 > kPhase2 ? kPhase1 : kPhase2;
+  static constexpr int kMain = kW2Off + kW2;
   static constexpr int kAux = kMain;  // barriers, slots, row arrays
   static constexpr int kAuxBytes = 256 + 128 * 4 * 2 + 2 * 4 * 128 * 4;
   static constexpr int kSmemBytes = 1024 + kMain + kAuxBytes;
@@ -301,12 +346,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       for (int p = 0; p < K1P; ++p)
         for (int h = 0; h < BN1 / kBox; ++h)
           tma_load_2d(sbase + Cfg::kA1 + p * BN1 * 128 + h * kBox * 128, &mapWin, p * 128, h * kBox, bw1);
-      // W_x goes where phase 1 lived: wait until the in_proj MMAs are done
-      if (mbar_wait(bd1, 0u, DEVFLAG_TIMEOUT_TMA)) {
-        mbar_arrive_expect_tx(bw2, (uint32_t)Cfg::kW2);
-        for (int p = 0; p < Cfg::kE1P; ++p)
-          tma_load_2d(sbase + Cfg::kW2Off + p * BN2 * 128, &mapWx, p * 128, 0, bw2);
-      }
+      mbar_arrive_expect_tx(bw2, (uint32_t)Cfg::kW2);
+      for (int p = 0; p < Cfg::kE1P; ++p)
+        tma_load_2d(sbase + Cfg::kW2Off + p * BN2 * 128, &mapWx, p * 128, 0, bw2);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -348,7 +390,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const long m = m0 + row;
     const bool live = m < P.M;
     // 1) codes of x into A1, deq_x into shared memory
-    quantize_rows_to_smem<Tx, 4 * K1P, 8>(reinterpret_cast<const Tx*>(P.x), d, m0, P.M, wi, lane,
+    quantize_rows_to_smem<Tx, 4 * K1P, 4>(reinterpret_cast<const Tx*>(P.x), d, m0, P.M, wi, lane,
                                           smem, deqx_s, P.deq_x, P.q_x, P.ld_qx);
     fence_proxy_async_smem();
     __syncwarp();
@@ -360,7 +402,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     constexpr int kSl = BN1 / 4;           // columns per worker
     const int cs = slice * kSl;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + cs;
-    const bool full = E == BN1;
+    constexpr bool full = true;  // the fused path runs with E == BN1
     int maxabs = 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < kSl; c0 += 32) {
@@ -407,10 +449,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         if (P.q_u != nullptr && live)
           *reinterpret_cast<uint4*>(P.q_u + m * P.ld_qu + col0 + hh * 16) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      float uv[32];
+      uint32_t uw[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) uv[j] = a[j] * c;
-      if (ok1) warp_store_block<0>(stg, uv, lane, P.u, nullptr, E, m0 + q * 32, col0, P.M, E);
+      for (int j = 0; j < 16; ++j) uw[j] = __byte_perm(r[2 * j], r[2 * j + 1], 0x5410);
+      if (ok1) warp_store_block_i16(reinterpret_cast<uint32_t*>(stg), uw, lane, P.u, E, m0 + q * 32, col0, P.M);
     }
     red_b[slice * 128 + row] = ss;
     fence_proxy_async_smem();
@@ -422,7 +464,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const float deq_u = (float)maxabs * c * (1.0f / sqrtf(c * c * (ss / (float)E) + kEpsNorm)) / 127.f;
     if (slice == 0) {
       dequ_s[row] = deq_u;
-      if (live) P.deq_u[m] = deq_u;
+      if (live) {
+        P.deq_u[m] = deq_u;
+        P.u_scale[m] = c;
+      }
     }
     // 3) x_proj epilogue (slice-0 workers hold whole rows): dt codes, B, C
     const bool ok2 = mbar_wait(bd2, 0u, DEVFLAG_TIMEOUT_EPI);
@@ -453,24 +498,49 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         P.deq_dt[m] = (float)mx * cdt * r_dt / 127.f;
       }
       const float cB = *P.s_B * deq_u, cC = *P.s_C * deq_u;
+      const bool fast = (R % 16 == 0) && (Ns == 16) && (P.ld_qdt == R);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN2; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(trow2 + c0, r);
         if (!live || !ok2) continue;
-        for (int j = 0; j < 32; ++j) {
-          const int col = c0 + j;
-          const int av = (int)r[j];
-          if (col < R) {
-            P.q_dt[m * P.ld_qdt + col] = (int8_t)(code_bits(i2f_exact(av), sg) & 0xff);
-          } else if (col < R + Ns) {
-            P.Bm[m * Ns + (col - R)] = i2f_exact(av) * cB;
-          } else if (col < R + 2 * Ns) {
-            P.Cm[m * Ns + (col - R - Ns)] = i2f_exact(av) * cC;
+        if (fast) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int col = c0 + hh * 16;
+            const uint32_t* rr = r + hh * 16;
+            if (col < R) {
+              uint32_t w[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                w[k] = pack4(code_bits(i2f_exact((int)rr[4 * k]), sg), code_bits(i2f_exact((int)rr[4 * k + 1]), sg),
+                             code_bits(i2f_exact((int)rr[4 * k + 2]), sg), code_bits(i2f_exact((int)rr[4 * k + 3]), sg));
+              *reinterpret_cast<uint4*>(P.q_dt + m * P.ld_qdt + col) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else if (col < R + 2 * Ns) {
+              const bool isB = col < R + Ns;
+              const float cf = isB ? cB : cC;
+              float4* dst = reinterpret_cast<float4*>((isB ? P.Bm : P.Cm) + m * Ns);
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4)
+                dst[v4] = make_float4(i2f_exact((int)rr[4 * v4]) * cf, i2f_exact((int)rr[4 * v4 + 1]) * cf,
+                                      i2f_exact((int)rr[4 * v4 + 2]) * cf, i2f_exact((int)rr[4 * v4 + 3]) * cf);
+            }
+          }
+        } else {
+          for (int j = 0; j < 32; ++j) {
+            const int col = c0 + j;
+            const int av = (int)r[j];
+            if (col < R) {
+              P.q_dt[m * P.ld_qdt + col] = (int8_t)(code_bits(i2f_exact(av), sg) & 0xff);
+            } else if (col < R + Ns) {
+              P.Bm[m * Ns + (col - R)] = i2f_exact(av) * cB;
+            } else if (col < R + 2 * Ns) {
+              P.Cm[m * Ns + (col - R - Ns)] = i2f_exact(av) * cC;
+            }
           }
         }
       }
-      if (live)
+      if (live && !fast)
         for (int col = R; col < P.ld_qdt; ++col) P.q_dt[m * P.ld_qdt + col] = 0;
     }
   }
@@ -571,7 +641,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const int slice = wi >> 2;
     const int row = q * 32 + lane;
     // 1) codes of y into A
-    quantize_rows_to_smem<float, 4 * KP, 2>(P.y, E, m0, P.M, wi, lane, smem, deq_s, P.deq_y, P.q_y,
+    quantize_rows_to_smem<float, 4 * KP, 4>(P.y, E, m0, P.M, wi, lane, smem, deq_s, P.deq_y, P.q_y,
                                             P.ld_qy);
     fence_proxy_async_smem();
     __syncwarp();

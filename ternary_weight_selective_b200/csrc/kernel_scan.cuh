@@ -20,6 +20,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels_rows.cuh"
 #include "ptx.cuh"
@@ -30,7 +31,8 @@ constexpr int kScanN = 16;   // d_state
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct ScanParams {
-  const void* u;          // [B, L, E]
+  const void* u;          // [B, L, E]  (int16 when u_scale is set: u = u_i16 * u_scale[token])
+  const float* u_scale;   // [B*L] nullable
   const void* delta_raw;  // [B, L, E] (unfused)
   const int8_t* q_dt;     // [B*L, ld_qdt] (fused)
   long ld_qdt;
@@ -132,9 +134,12 @@ struct ScanStage {
   static constexpr int kBC = kScanChunk * kScanN * 4;
   static constexpr int kQ = FUSED ? kScanChunk * 128 : 0;  // dt codes, row pitch 128 B
   static constexpr int kDeq = FUSED ? kScanChunk * 4 : 0;
+  // int16 u (exact in_proj accumulators) comes with a per-token scale
+  static constexpr bool kI16 = std::is_same<Tu, int16_t>::value;
+  static constexpr int kUs = kI16 ? kScanChunk * 4 : 0;
   static constexpr int oU = 0, oD = oU + kU, oB = oD + kD, oC = oB + kBC, oQ = oC + kBC,
-                       oDeq = oQ + kQ;
-  static constexpr int kBytes = oDeq + kDeq;
+                       oDeq = oQ + kQ, oUs = oDeq + kDeq;
+  static constexpr int kBytes = oUs + kUs;
 };
 
 // Selective scan.  A CTA of 128 threads owns CE = 128*NPT/16 channels of one
@@ -212,14 +217,23 @@ __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
       for (int t = tid; t < kScanChunk; t += 128)
         cp_async4(sb + St::oDeq + t * 4, P.deq_dt + tok0 + min(t0 + t, L - 1), (t0 + t < L) ? 4 : 0);
     }
+    if constexpr (St::kUs > 0) {
+      for (int t = tid; t < kScanChunk; t += 128)
+        cp_async4(sb + St::oUs + t * 4, P.u_scale + tok0 + min(t0 + t, L - 1), (t0 + t < L) ? 4 : 0);
+    }
   };
 
-  float A2[NPT], h[NPT];
+  // states and decay rates as pairs: the recurrence runs on the paired
+  // fp32 pipe (fma.rn.f32x2 / mul.rn.f32x2), two states per instruction
+  float2 A2[NPT / 2], h[NPT / 2];
 #pragma unroll
-  for (int j = 0; j < NPT; ++j) {
-    const int n = g * NPT + j;
-    A2[j] = ch_ok ? P.A[(long)e * kScanN + n] * kLog2e : 0.f;
-    h[j] = (ch_ok && P.h0 != nullptr) ? P.h0[((long)b * E + e) * kScanN + n] : 0.f;
+  for (int j = 0; j < NPT / 2; ++j) {
+    const int n = g * NPT + 2 * j;
+    A2[j] = ch_ok ? make_float2(P.A[(long)e * kScanN + n] * kLog2e, P.A[(long)e * kScanN + n + 1] * kLog2e)
+                  : make_float2(0.f, 0.f);
+    h[j] = (ch_ok && P.h0 != nullptr)
+               ? make_float2(P.h0[((long)b * E + e) * kScanN + n], P.h0[((long)b * E + e) * kScanN + n + 1])
+               : make_float2(0.f, 0.f);
   }
   const float Dv = ch_ok ? P.D[e] : 0.f;
   const float bias = ch_ok ? P.bias[e] : 0.f;
@@ -254,7 +268,11 @@ __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
 #pragma unroll
     for (int i = 0; i < SPL; ++i) {
       const int tl = i * TPC + g;
-      const float uv = load_as_float(u_s + tl * CE + c);
+      float uv;
+      if constexpr (St::kUs > 0)
+        uv = i2f_exact((int)u_s[tl * CE + c]) * reinterpret_cast<const float*>(sp + St::oUs)[tl];
+      else
+        uv = load_as_float(u_s + tl * CE + c);
       float z;
       if constexpr (FUSED) {
         const int4* qv = reinterpret_cast<const int4*>(sp + St::oQ + tl * 128);
@@ -287,39 +305,45 @@ __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
     // tl+1 are issued before the state updates of step tl, so each exp2 has
     // a full step of independent work between it and its use.
     float ys[SPL];
-    float a_cur[NPT];
+    float2 a_cur[NPT / 2];
+    {
+      const float2 d2 = make_float2(dls[0], dls[0]);
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) a_cur[j] = ex2_approx(dls[0] * A2[j]);
+      for (int j = 0; j < NPT / 2; ++j) {
+        const float2 x = __fmul2_rn(d2, A2[j]);
+        a_cur[j] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+    }
     float yp[TPC];
 #pragma unroll
     for (int tl = 0; tl < kScanChunk; ++tl) {
-      float a_nxt[NPT];
+      float2 a_nxt[NPT / 2];
       if (tl + 1 < kScanChunk) {
+        const float2 d2 = make_float2(dls[tl + 1], dls[tl + 1]);
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) a_nxt[j] = ex2_approx(dls[tl + 1] * A2[j]);
+        for (int j = 0; j < NPT / 2; ++j) {
+          const float2 x = __fmul2_rn(d2, A2[j]);
+          a_nxt[j] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        }
       }
       const float4* Bp = reinterpret_cast<const float4*>(B_s + tl * kScanN + g * NPT);
       const float4* Cp = reinterpret_cast<const float4*>(C_s + tl * kScanN + g * NPT);
-      const float du_s = dus[tl];
-      float acc0 = 0.f, acc1 = 0.f;
+      const float2 du2 = make_float2(dus[tl], dus[tl]);
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int v = 0; v < NPT / 4; ++v) {
         const float4 b4 = Bp[v];
         const float4 c4 = Cp[v];
-        h[4 * v + 0] = fmaf(a_cur[4 * v + 0], h[4 * v + 0], du_s * b4.x);
-        h[4 * v + 1] = fmaf(a_cur[4 * v + 1], h[4 * v + 1], du_s * b4.y);
-        h[4 * v + 2] = fmaf(a_cur[4 * v + 2], h[4 * v + 2], du_s * b4.z);
-        h[4 * v + 3] = fmaf(a_cur[4 * v + 3], h[4 * v + 3], du_s * b4.w);
-        acc0 = fmaf(c4.x, h[4 * v + 0], acc0);
-        acc1 = fmaf(c4.y, h[4 * v + 1], acc1);
-        acc0 = fmaf(c4.z, h[4 * v + 2], acc0);
-        acc1 = fmaf(c4.w, h[4 * v + 3], acc1);
+        h[2 * v] = __ffma2_rn(a_cur[2 * v], h[2 * v], __fmul2_rn(du2, make_float2(b4.x, b4.y)));
+        h[2 * v + 1] = __ffma2_rn(a_cur[2 * v + 1], h[2 * v + 1], __fmul2_rn(du2, make_float2(b4.z, b4.w)));
+        acc = __ffma2_rn(make_float2(c4.x, c4.y), h[2 * v], acc);
+        acc = __ffma2_rn(make_float2(c4.z, c4.w), h[2 * v + 1], acc);
       }
-      yp[tl % TPC] = acc0 + acc1;
+      yp[tl % TPC] = acc.x + acc.y;
       if (tl % TPC == TPC - 1) ys[tl / TPC] = reduce_scatter<TPC>(yp, g) + Du[tl / TPC];
       if (tl + 1 < kScanChunk) {
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) a_cur[j] = a_nxt[j];
+        for (int j = 0; j < NPT / 2; ++j) a_cur[j] = a_nxt[j];
       }
     }
     if (ch_ok) {
@@ -332,7 +356,10 @@ __global__ void __launch_bounds__(128) selective_scan_kernel(ScanParams P) {
   }
   if (P.h_last != nullptr && ch_ok) {
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) P.h_last[((long)b * E + e) * kScanN + g * NPT + j] = h[j];
+    for (int j = 0; j < NPT / 2; ++j) {
+      P.h_last[((long)b * E + e) * kScanN + g * NPT + 2 * j] = h[j].x;
+      P.h_last[((long)b * E + e) * kScanN + g * NPT + 2 * j + 1] = h[j].y;
+    }
   }
 }
 

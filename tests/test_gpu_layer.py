@@ -63,7 +63,14 @@ def a8_stage_checks(env, x, lw, ws, dl, out_gpu, dtype):
     q_x = g(v.q_x, torch.int8, (T, v.ld_qx))
     assert np.array_equal(q_x[:, :d], st["q_x"]) and not q_x[:, d:].any()
     assert rel_err(g(v.deq_x, torch.float32, (T,)), st["deq_x"]) <= 1e-5
-    u = g(v.u, torch.float32, (T, E))
+    if v.u_dtype == abi.I16:
+        # fused kernels: u kept as the exact int16 in_proj accumulators and a
+        # per-token scale
+        u_i = g(v.u, torch.int16, (T, E)).astype(np.int64)
+        assert np.array_equal(u_i, st["acc_in"])
+        u = u_i * g(v.u_scale, torch.float32, (T,))[:, None].astype(np.float64)
+    else:
+        u = g(v.u, torch.float32, (T, E))
     assert rel_err(u, st["u"]) <= 1e-5
     q_u = g(v.q_u, torch.int8, (T, v.ld_qu))
     assert np.array_equal(q_u[:, :E], st["q_u"])
