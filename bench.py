@@ -44,6 +44,25 @@ SM_COUNT = 148
 SM_MAX_MHZ = 1965.0
 
 
+def recorded_traffic(profile_md: str, source: str):
+    """DRAM bytes per launch recorded by an ncu capture summarised in
+    profiles/, or None when the kernel source has changed since."""
+    import hashlib
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile_md)).read()
+        src = open(os.path.join(ROOT, "ternary_weight_selective_b200", "csrc", source), "rb").read()
+    except OSError:
+        return None
+    sha = hashlib.sha256(src).hexdigest()[:16]
+    rec_sha = traffic = None
+    for line in text.splitlines():
+        if line.startswith("kernel_source_sha256_16:"):
+            rec_sha = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = int(line.split(":", 1)[1].strip())
+    return traffic if rec_sha == sha else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -169,7 +188,11 @@ def run_ours(args):
         return evs
 
     def timed(prepared: bool, sample_clocks: bool):
-        """K forwards (CUDA-graph replays); returns per-step ms and per-kernel ms."""
+        """K forwards as CUDA-graph replays.  The step time is taken from a
+        graph of G x (L2 flush + forward) with no event inside, minus a graph
+        of G x (L2 flush) alone; a second graph with an event before every
+        kernel (recorded by the library) gives the per-kernel breakdown
+        (those intervals also contain the event nodes' own cost)."""
         for d_l in dl:
             if prepared:
                 d_l.prepare()
@@ -180,40 +203,63 @@ def run_ours(args):
         nl = abi.bitssm_forward_launches(dl[0].layer, act)
         per_step = n_layers * (nl + 1)
 
-        def step(evs):
-            """One forward; evs: (nl + 1) events per layer, recorded by the
-            library before every kernel and after the last."""
+        def forward(evs=None):
             st = torch.cuda.current_stream()
             h_in = xd
             for li, d_l in enumerate(dl):
-                e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
-                abi.bitssm_forward_timed(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B,
-                                         L, dtype, act, ws.addr, nbytes,
-                                         [ev.cuda_event for ev in e], st)
+                res = h_in if n_layers > 1 else None
+                if evs is None:
+                    abi.bitssm_forward(d_l.layer, h_in, out, res, B, L, dtype, act, ws.addr,
+                                       nbytes, st)
+                else:
+                    e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
+                    abi.bitssm_forward_timed(d_l.layer, h_in, out, res, B, L, dtype, act,
+                                             ws.addr, nbytes, [ev.cuda_event for ev in e], st)
                 h_in = out
 
         # eager warm-up (also sets the kernels' shared-memory attributes)
-        warm = new_events(per_step)
         for _ in range(args.warmup):
             flush.zero_()
-            step(warm)
+            forward()
         torch.cuda.synchronize()
-        # The timed steps run as CUDA-graph replays (host launch cost out of
-        # the device timeline): one graph holds G x (L2 flush + forward).
         G = max(1, min(args.steps, 100))
         R = (args.steps + G - 1) // G
         gevents = [new_events(per_step) for _ in range(G)]
         torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream()
-        cap.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.graph(graph, stream=cap):
-            for i in range(G):
-                flush.zero_()
-                step(gevents[i])
-        torch.cuda.synchronize()
-        graph.replay()  # one untimed replay
-        torch.cuda.synchronize()
+
+        def capture(body):
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream()
+            cap.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(G):
+                    body(i)
+            torch.cuda.synchronize()
+            g.replay()  # one untimed replay
+            torch.cuda.synchronize()
+            return g
+
+        def body_plain(i):
+            flush.zero_()
+            forward()
+
+        def body_flush(i):
+            flush.zero_()
+
+        def body_events(i):
+            flush.zero_()
+            forward(gevents[i])
+
+        g_plain, g_flush, g_ev = capture(body_plain), capture(body_flush), capture(body_events)
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def replay_ms(g):
+            ea.record()
+            g.replay()
+            eb.record()
+            torch.cuda.synchronize()
+            return ea.elapsed_time(eb)
+
         sampler = None
         if sample_clocks and rank == 0:
             props = torch.cuda.get_device_properties(local)
@@ -221,36 +267,40 @@ def run_ours(args):
             sampler = ClockSampler(gpu_id)
             sampler.start()
             time.sleep(0.3)
-        step_ms, kern_ms = [], [[0.0] * nl for _ in range(n_layers)]
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         t_wall = time.perf_counter()
+        plain_ms = flush_ms = 0.0
         for _ in range(R):
-            graph.replay()
-            torch.cuda.synchronize()
-            for evs in gevents:
-                tot = 0.0
-                for li in range(n_layers):
-                    e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
-                    for i in range(nl):
-                        kern_ms[li][i] += e[i].elapsed_time(e[i + 1])
-                    tot += e[0].elapsed_time(e[nl])
-                step_ms.append(tot)
+            plain_ms += replay_ms(g_plain)
+            flush_ms += replay_ms(g_flush)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
         if world > 1:
             dist.barrier()
         clocks = sampler.stop() if sampler is not None else None
-        del graph
-        total_ms = sum(step_ms)
+        kern_ms = [[0.0] * nl for _ in range(n_layers)]
+        ev_step_ms = 0.0
+        for _ in range(R):
+            g_ev.replay()
+            torch.cuda.synchronize()
+            for evs in gevents:
+                for li in range(n_layers):
+                    e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
+                    for i in range(nl):
+                        kern_ms[li][i] += e[i].elapsed_time(e[i + 1])
+                    ev_step_ms += e[0].elapsed_time(e[nl])
+        del g_plain, g_flush, g_ev
+        K = G * R
+        total_ms = plain_ms - flush_ms
         if world > 1:
             t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             total_ms = float(t.item())
-        K = G * R
         return dict(ms=total_ms / K, kern_ms=kern_ms, nl=nl, K=K, G=G, R=R, t_wall=t_wall,
-                    clocks=clocks, ws=ws, nbytes=nbytes)
+                    clocks=clocks, ws=ws, nbytes=nbytes, ev_step_ms=ev_step_ms / K,
+                    flush_ms=flush_ms / K)
 
     # the hot path: weights expanded once (bitssm_prepare_weights), then every
     # forward of the timed region runs every stage on fresh activations
@@ -323,7 +373,8 @@ def run_ours(args):
         names = names[1:]
     avg_kernel_ms = [sum(kern_ms[li][i] for li in range(n_layers)) / (args.steps * n_layers)
                      for i in range(nl)]
-    share = {names[i]: round(avg_kernel_ms[i] / (ms_per_step / n_layers), 4) for i in range(nl)}
+    ev_layer_ms = main["ev_step_ms"] / n_layers
+    share = {names[i]: round(avg_kernel_ms[i] / ev_layer_ms, 4) for i in range(nl)}
     dom = max(range(nl), key=lambda i: avg_kernel_ms[i])
     peaks, peak_kind = load_peaks()
     sm_max = (clocks or {}).get("sm_max_mhz") or peaks.get("sm_max_mhz", SM_MAX_MHZ)
@@ -339,7 +390,9 @@ def run_ours(args):
                 "achieved": round(achieved, 4), "peak": round(peak, 4),
                 "frac": round(achieved / peak, 4),
                 "peak_source": f"{MUFU_EX2_PER_CLK_PER_SM} ex2/clk/SM x {SM_COUNT} SMs x {sm_max:.0f} MHz",
-                "traffic": None,
+                "traffic": (recorded_traffic("selective_scan_trissm.md", "kernel_scan.cuh")
+                            if wl.name == "trissm" else None),
+                "traffic_note": "ncu dram__bytes_read+write per launch (cold L2); y's writes are still dirty in L2 when the kernel ends",
                 "hbm_achieved_gbs": round(hbm_bytes / t_s / 1e9, 1),
                 "hbm_frac": round(hbm_bytes / t_s / 1e9 / peaks["hbm_gbs"], 4),
                 "hbm_peak_source": f"{peak_kind} hbm_gbs"}
@@ -364,7 +417,7 @@ def run_ours(args):
                    "l2": "flushed before every timed step (256 MiB write, outside the events)"},
         "roofline": roof,
         "kernel_share": share,
-        "kernel_avg_us": {names[i]: round(avg_kernel_ms[i] * 1e3, 2) for i in range(nl)},
+        "kernel_avg_us_instrumented": {names[i]: round(avg_kernel_ms[i] * 1e3, 2) for i in range(nl)},
         "weights": "expanded once before the timed region (bitssm_prepare_weights)",
         "value_with_per_call_weight_expansion": round(T * world / (unprep["ms"] / 1e3), 1),
         "layer_hbm_gbs_algorithmic": round(layer_gbs, 1),
@@ -373,7 +426,11 @@ def run_ours(args):
         "gpu_launches": args.steps * n_layers * nl,
         "clocks": clocks,
         "wall_s_timed_region": round(t_wall, 4),
-        "timing": f"{R} replays of a CUDA graph of {G} x (L2 flush + forward); per-kernel CUDA events inside the graph",
+        "timing": (f"{R} replays each of CUDA graphs of {G} x (L2 flush + forward) and {G} x (L2 flush); "
+                   "step = difference / G; per-kernel times from a third graph with an event before "
+                   "every kernel (its intervals include the event nodes' own cost)"),
+        "instrumented_ms_per_step": round(main["ev_step_ms"], 5),
+        "flush_ms": round(main["flush_ms"], 5),
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)

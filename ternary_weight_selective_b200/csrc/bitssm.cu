@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -262,12 +263,25 @@ int launch_scan_t(const ScanParams& P, cudaStream_t st) {
 
 // States per thread: 16 (one thread per channel, no exchange) when there are
 // enough channels to give every SM sub-partition ~1.5 warps, else 8 or 4.
+// Tuning override of the states-per-thread choice (4, 8 or 16), read once
+// from the environment variable BITSSM_SCAN_NPT; 0 = automatic.
+int scan_npt_override() {
+  static const int v = [] {
+    const char* e = std::getenv("BITSSM_SCAN_NPT");
+    const int n = e ? std::atoi(e) : 0;
+    return (n == 4 || n == 8 || n == 16) ? n : 0;
+  }();
+  return v;
+}
+
 template <bool FUSED, int RV, typename Tu, typename Td, typename Ty>
 int launch_scan_rv(const ScanParams& P, cudaStream_t st) {
   const long channels = (long)P.B * P.E;
   const long want = (long)num_sms() * 4 * 48;
-  if (channels >= want) return launch_scan_t<16, FUSED, RV, Tu, Td, Ty>(P, st);
-  if (channels * 2 >= want) return launch_scan_t<8, FUSED, RV, Tu, Td, Ty>(P, st);
+  int npt = channels >= want ? 16 : (channels * 2 >= want ? 8 : 4);
+  if (scan_npt_override() != 0) npt = scan_npt_override();
+  if (npt == 16) return launch_scan_t<16, FUSED, RV, Tu, Td, Ty>(P, st);
+  if (npt == 8) return launch_scan_t<8, FUSED, RV, Tu, Td, Ty>(P, st);
   return launch_scan_t<4, FUSED, RV, Tu, Td, Ty>(P, st);
 }
 
