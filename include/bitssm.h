@@ -162,6 +162,31 @@ int bitlinear_forward(const bitssm_tw* w, const void* x, int M, int x_dtype, voi
                       int act_mode, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------
+ * bitlinear_forward without a caller workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves, for example an operator running inside a host
+ * framework whose allocator must own every device byte, code held to a
+ * memory budget fixed at start-up, or a latency-critical path where an
+ * allocation and its implicit synchronisation are not acceptable.
+ *
+ * Same arguments, results and errors as bitlinear_forward, minus ws and
+ * ws_bytes: the scratch is a fixed array of BITSSM_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) inside the library, present on every GPU that loads the library
+ * until the process exits.  A shape whose bitlinear_workspace_size exceeds
+ * that returns BITSSM_ERR_WORKSPACE, with the sizes in bitssm_last_error().
+ * The call allocates nothing (no cudaMalloc, no library allocator).
+ *  - The first call on a device looks up the array's device address on the
+ *    current device; make that first call before any stream capture.
+ *  - Every call shares the one array: calls whose work overlaps on the GPU
+ *    (different streams, or concurrent host threads) race and corrupt each
+ *    other; serialise them, e.g. on one stream.  Nothing in the array needs
+ *    to start at zero; each call rewrites what it reads.
+ * --------------------------------------------------------------------- */
+#define BITSSM_NOALLOC_SCRATCH_BYTES (16u << 20)
+int bitlinear_forward_noalloc(const bitssm_tw* w, const void* x, int M, int x_dtype, void* y,
+                              int y_dtype, int act_mode, void* stream);
+
+/* ---------------------------------------------------------------------
  * Selective scan (the BitSSM recurrence; TriSSM README caption and
  * "Repository structure": the recurrence is evaluated with a parallel
  * associative scan).  For every batch b, channel e, state n, step t:

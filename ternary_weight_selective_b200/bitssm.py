@@ -85,6 +85,7 @@ _SIGS = {
     "bitssm_pack_ternary": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "bitlinear_workspace_size": (_i, [_P_TW, _i, _i, ctypes.POINTER(_sz)]),
     "bitlinear_forward": (_i, [_P_TW, _vp, _i, _i, _vp, _i, _i, _vp, _sz, _vp]),
+    "bitlinear_forward_noalloc": (_i, [_P_TW, _vp, _i, _i, _vp, _i, _i, _vp]),
     "selective_scan_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                     _i, _i, _i, _i, _i, _vp]),
     "bitssm_workspace_size": (_i, [_P_LAYER, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
@@ -172,6 +173,16 @@ def bitlinear_forward(w: bitssm_tw, x, M, x_dtype, y, y_dtype, act_mode, ws, ws_
     _check(_lib.bitlinear_forward(ctypes.byref(w), _ptr(x), M, x_dtype, _ptr(y), y_dtype,
                                   act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitlinear_forward")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def bitlinear_forward_noalloc(w: bitssm_tw, x, M, x_dtype, y, y_dtype, act_mode, stream=None):
+    """bitlinear_forward on the library's built-in scratch array, for callers
+    that cannot allocate device memory (see include/bitssm.h)."""
+    _check(_lib.bitlinear_forward_noalloc(ctypes.byref(w), _ptr(x), M, x_dtype, _ptr(y), y_dtype,
+                                          act_mode, _stream(stream)), "bitlinear_forward_noalloc")
 
 
 def selective_scan_forward(u, delta_raw, delta_bias, A, Bm, Cm, D, h0, y, h_last,

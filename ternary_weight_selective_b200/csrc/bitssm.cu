@@ -28,7 +28,7 @@ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // Name of the last CUDA error this library saw on this thread.
-thread_local char g_last_error[160] = "no error";
+thread_local char g_last_error[256] = "no error";
 void note_cuda_error(cudaError_t e) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
                 cudaGetErrorString(e));
@@ -796,6 +796,12 @@ int check_layer_args(const bitssm_layer* p, int B, int L, int dtype, int act_mod
 }
 
 }  // namespace
+
+// Lets other translation units of this library set the message returned by
+// bitssm_last_error() for a status they return.
+void set_last_error_message(const char* msg) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+}
 }  // namespace bitssm
 
 using namespace bitssm;
