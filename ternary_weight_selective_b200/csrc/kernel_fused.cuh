@@ -30,7 +30,6 @@ namespace bitssm {
 
 constexpr int kFusedWorkers = 16;
 constexpr int kFusedThreads = 64 + 32 * kFusedWorkers;
-constexpr int kStageFloats = 32 * 36;  // one warp's 32 x 32 fp32 transpose buffer (padded rows)
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -42,78 +41,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ uint32_t sw128_off(int row, int kbyte) {
   const int kb = kbyte & 127;
   return (uint32_t)((kbyte >> 7) * (128 * 128) + row * 128 + ((((kb >> 4) ^ (row & 7)) << 4) | (kb & 15)));
-}
-
-// One warp stores a 32-row x 32-column fp32 block, row i held by lane i in
-// v[0..31], through its shared buffer: the lanes first write their rows,
-// then each store instruction covers 4 (fp32) or 8 (bf16) rows of 128 / 64
-// contiguous bytes.  out row r of the block is out + (row0 + r) * ld + col0;
-// rows >= M and columns >= ncols are skipped; residual (nullable) is added.
-template <int OUT_BF16>
-__device__ __forceinline__ void warp_store_block(float* sbuf, const float (&v)[32], int lane,
-                                                 void* out, const void* residual, long ld,
-                                                 long row0, int col0, long M, int ncols) {
-  float4* srow = reinterpret_cast<float4*>(sbuf + lane * 36);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) srow[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-  __syncwarp();
-  if constexpr (!OUT_BF16) {
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int r = it * 4 + (lane >> 3);
-      const int cc = (lane & 7) * 4;
-      const long m = row0 + r;
-      if (m < M && col0 + cc < ncols) {
-        float4 val = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc);
-        float* dst = reinterpret_cast<float*>(out) + m * ld + col0 + cc;
-        if (col0 + cc + 4 <= ncols) {
-          if (residual != nullptr) {
-            const float4 rr = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(residual) + m * ld + col0 + cc);
-            val.x += rr.x; val.y += rr.y; val.z += rr.z; val.w += rr.w;
-          }
-          *reinterpret_cast<float4*>(dst) = val;
-        } else {
-          const float vv[4] = {val.x, val.y, val.z, val.w};
-          for (int j = 0; col0 + cc + j < ncols; ++j)
-            dst[j] = vv[j] + (residual ? reinterpret_cast<const float*>(residual)[m * ld + col0 + cc + j] : 0.f);
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int r = it * 8 + (lane >> 2);
-      const int cc = (lane & 3) * 8;
-      const long m = row0 + r;
-      if (m < M && col0 + cc < ncols) {
-        const float4 a = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc);
-        const float4 b = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc + 4);
-        float vv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out) + m * ld + col0 + cc;
-        if (col0 + cc + 8 <= ncols) {
-          if (residual != nullptr) {
-            const uint4 rr = *reinterpret_cast<const uint4*>(
-                reinterpret_cast<const __nv_bfloat16*>(residual) + m * ld + col0 + cc);
-            const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              vv[2 * k] += __uint_as_float(w[k] << 16);
-              vv[2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
-            }
-          }
-          *reinterpret_cast<uint4*>(dst) =
-              make_uint4(pack_bf16x2(vv[0], vv[1]), pack_bf16x2(vv[2], vv[3]),
-                         pack_bf16x2(vv[4], vv[5]), pack_bf16x2(vv[6], vv[7]));
-        } else {
-          for (int j = 0; col0 + cc + j < ncols; ++j) {
-            const float rres = residual ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(residual)[m * ld + col0 + cc + j]) : 0.f;
-            dst[j] = __float2bfloat16_rn(vv[j] + rres);
-          }
-        }
-      }
-    }
-  }
-  __syncwarp();
 }
 
 // One warp stores a 32-row x 32-column block of int16 values, row i held

@@ -167,6 +167,81 @@ __device__ __forceinline__ void add_residual16(const void* base, long idx, int d
   }
 }
 
+constexpr int kStageFloats = 32 * 36;  // one warp's 32 x 32 fp32 transpose buffer (padded rows)
+
+// One warp stores a 32-row x 32-column fp32 block, row i held by lane i in
+// v[0..31], through its shared buffer: the lanes first write their rows,
+// then each store instruction covers 4 (fp32) or 8 (bf16) rows of 128 / 64
+// contiguous bytes.  out row r of the block is out + (row0 + r) * ld + col0;
+// rows >= M and columns >= ncols are skipped; residual (nullable) is added.
+template <int OUT_BF16>
+__device__ __forceinline__ void warp_store_block(float* sbuf, const float (&v)[32], int lane,
+                                                 void* out, const void* residual, long ld,
+                                                 long row0, int col0, long M, int ncols) {
+  float4* srow = reinterpret_cast<float4*>(sbuf + lane * 36);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) srow[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  __syncwarp();
+  if constexpr (!OUT_BF16) {
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int r = it * 4 + (lane >> 3);
+      const int cc = (lane & 7) * 4;
+      const long m = row0 + r;
+      if (m < M && col0 + cc < ncols) {
+        float4 val = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc);
+        float* dst = reinterpret_cast<float*>(out) + m * ld + col0 + cc;
+        if (col0 + cc + 4 <= ncols) {
+          if (residual != nullptr) {
+            const float4 rr = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(residual) + m * ld + col0 + cc);
+            val.x += rr.x; val.y += rr.y; val.z += rr.z; val.w += rr.w;
+          }
+          *reinterpret_cast<float4*>(dst) = val;
+        } else {
+          const float vv[4] = {val.x, val.y, val.z, val.w};
+          for (int j = 0; col0 + cc + j < ncols; ++j)
+            dst[j] = vv[j] + (residual ? reinterpret_cast<const float*>(residual)[m * ld + col0 + cc + j] : 0.f);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int r = it * 8 + (lane >> 2);
+      const int cc = (lane & 3) * 8;
+      const long m = row0 + r;
+      if (m < M && col0 + cc < ncols) {
+        const float4 a = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc);
+        const float4 b = *reinterpret_cast<const float4*>(sbuf + r * 36 + cc + 4);
+        float vv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out) + m * ld + col0 + cc;
+        if (col0 + cc + 8 <= ncols) {
+          if (residual != nullptr) {
+            const uint4 rr = *reinterpret_cast<const uint4*>(
+                reinterpret_cast<const __nv_bfloat16*>(residual) + m * ld + col0 + cc);
+            const uint32_t w[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              vv[2 * k] += __uint_as_float(w[k] << 16);
+              vv[2 * k + 1] += __uint_as_float(w[k] & 0xffff0000u);
+            }
+          }
+          *reinterpret_cast<uint4*>(dst) =
+              make_uint4(pack_bf16x2(vv[0], vv[1]), pack_bf16x2(vv[2], vv[3]),
+                         pack_bf16x2(vv[4], vv[5]), pack_bf16x2(vv[6], vv[7]));
+        } else {
+          for (int j = 0; col0 + cc + j < ncols; ++j) {
+            const float rres = residual ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(residual)[m * ld + col0 + cc + j]) : 0.f;
+            dst[j] = __float2bfloat16_rn(vv[j] + rres);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
+
 // int8 x ternary GEMM (A8).  Warp 0 lane 0: TMA producer; warp 1: TMEM
 // owner and MMA issuer (lane 0); warps 2 .. 2+4*CSPLIT-1: epilogue, warp w
 // on the 32 TMEM lanes (rows) of quadrant w % 4 and on column slice
@@ -477,10 +552,18 @@ struct GsConfig {
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOffset = STAGES * kStageBytes;
+  // Ring of per-group scale rows (BN floats each), filled by the producer
+  // with the group's first panel.  The producer runs at most STAGES panels
+  // (STAGES/2 groups) ahead of the MMAs, which run at most two groups ahead
+  // of the epilogue, so this many slots are never overwritten while read.
+  static constexpr int kScaleSlots = 8;
+  static_assert(kScaleSlots >= STAGES / 2 + 3, "scale ring");
+  static constexpr int kScaleOffset = STAGES * kStageBytes;
+  static constexpr int kBarOffset = kScaleOffset + kScaleSlots * BN * 4;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
   static constexpr int kHalf = BN / 2;  // columns per epilogue warp
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(8 * kStageFloats * 4 <= STAGES * kStageBytes, "output staging");
 };
 
 template <int BN, int STAGES, int EPI>
@@ -532,15 +615,23 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0 && lane == 0) {
     constexpr uint32_t kTx = Cfg::kABytes + Cfg::kBBytes;
+    constexpr uint32_t kScaleRow = BN * 4;
     for (int p = 0; p < num_panels; ++p) {
       const int s = p % STAGES;
       const uint32_t ph = (uint32_t)(p / STAGES) & 1u;
       if (p >= STAGES && !mbar_wait(empty_bar(s), ph ^ 1u, DEVFLAG_TIMEOUT_TMA)) break;
       const uint32_t sa = sbase + s * Cfg::kStageBytes;
-      mbar_arrive_expect_tx(full_bar(s), kTx);
+      const bool first = (p % kPanelsPerGroup) == 0;
+      mbar_arrive_expect_tx(full_bar(s), kTx + (first ? kScaleRow : 0u));
       const int kc = p * kPanel;
       tma_load_2d(sa, &mapA, kc, m0, full_bar(s));
       tma_load_2d(sa + Cfg::kABytes, &mapW, kc, n0, full_bar(s));
+      if (first) {
+        // this group's scales for the tile's columns: s_t[g][n0 .. n0+BN)
+        const int grp = p / kPanelsPerGroup;
+        bulk_load_1d(sbase + Cfg::kScaleOffset + (grp % Cfg::kScaleSlots) * kScaleRow,
+                     P.s_t + (long)grp * P.ld_s + n0, kScaleRow, full_bar(s));
+      }
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t kIdesc = umma_idesc(1u, 1u, 128u, (uint32_t)BN);
@@ -587,15 +678,22 @@ __global__ void __launch_bounds__(320, 1)
       ok = mbar_wait(pfull_bar(buf), (uint32_t)(g >> 1) & 1u, DEVFLAG_TIMEOUT_EPI);
       if (!ok) break;
       tc_fence_after();
-      const float* sg = P.s_t + (long)g * P.ld_s + n0 + c_base;
+      // the group's scale row landed with its first panel, before the MMAs
+      const float4* s4 = reinterpret_cast<const float4*>(
+          smem + Cfg::kScaleOffset + (g % Cfg::kScaleSlots) * (BN * 4) + c_base * 4);
+      // columns per TMEM round trip: 16 with 128 accumulators per thread
+      // (register budget), else 32
+      constexpr int kLd = Cfg::kHalf >= 128 ? 16 : 32;
 #pragma unroll
-      for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(trow + buf * 256 + c0, r);
-        const float4* s4 = reinterpret_cast<const float4*>(sg + c0);
+      for (int c0 = 0; c0 < Cfg::kHalf; c0 += kLd) {
+        uint32_t r[kLd];
+        if constexpr (kLd == 16)
+          tmem_ld16(trow + buf * 256 + c0, r);
+        else
+          tmem_ld32(trow + buf * 256 + c0, r);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 sv = __ldg(s4 + v);
+        for (int v = 0; v < kLd / 4; ++v) {
+          const float4 sv = s4[c0 / 4 + v];
           acc[c0 + 4 * v + 0] = fmaf(sv.x, __uint_as_float(r[4 * v + 0]), acc[c0 + 4 * v + 0]);
           acc[c0 + 4 * v + 1] = fmaf(sv.y, __uint_as_float(r[4 * v + 1]), acc[c0 + 4 * v + 1]);
           acc[c0 + 4 * v + 2] = fmaf(sv.z, __uint_as_float(r[4 * v + 2]), acc[c0 + 4 * v + 2]);
@@ -606,39 +704,52 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(pempty_bar(buf));
     }
-    if (ok && live) {
-      const float rs = P.row_scale != nullptr ? P.row_scale[m] : 1.0f;
-      if constexpr (EPI == EPI_STORE) {
-        const int ncols = min(BN, P.N - n0);
-#pragma unroll
-        for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
-          const int col = c_base + c0;
-          if (col >= ncols) break;
-          const int valid = min(16, ncols - col);
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = acc[c0 + j] * rs;
-          const long idx = (long)m * P.ld_out + n0 + col;
-          if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
-          store16(P.out, idx, P.out_dtype, v, valid);
-        }
-      } else if constexpr (EPI == EPI_ROWSS) {
+    // STORE / ROWSS with a float or bf16 output: coalesced stores through a
+    // per-warp transpose buffer in the (now idle) pipeline stages.  Every
+    // lane takes part (rows >= M are skipped inside the store).
+    if constexpr (EPI == EPI_STORE || EPI == EPI_ROWSS) {
+      const int odt = EPI == EPI_ROWSS ? 1 : P.out_dtype;
+      if (ok && odt != 2) {
+        const float rs = (live && P.row_scale != nullptr) ? P.row_scale[m] : 1.0f;
+        float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * kStageFloats;
+        const void* res = EPI == EPI_STORE ? P.residual : nullptr;
         const int ncols = min(BN, P.N - n0);
         float ss = 0.f;
 #pragma unroll
-        for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
-          const int col = c_base + c0;
-          if (col >= ncols) break;
-          const int valid = min(16, ncols - col);
-          float v[16];
+        for (int c0 = 0; c0 < Cfg::kHalf; c0 += 32) {
+          float v[32];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 32; ++j) {
             v[j] = acc[c0 + j] * rs;
-            if (j < valid) ss = fmaf(v[j], v[j], ss);
+            if (EPI == EPI_ROWSS && c_base + c0 + j < ncols) ss = fmaf(v[j], v[j], ss);
           }
-          store16(P.out, (long)m * P.ld_out + n0 + col, 1, v, valid);
+          if (odt == 1)
+            warp_store_block<1>(stg, v, lane, P.out, res, P.ld_out, m0 + q * 32, n0 + c_base + c0, P.M, P.N);
+          else
+            warp_store_block<0>(stg, v, lane, P.out, res, P.ld_out, m0 + q * 32, n0 + c_base + c0, P.M, P.N);
         }
-        P.ss_part[(long)m * (2 * gridDim.y) + 2 * blockIdx.y + half] = ss;
+        if (EPI == EPI_ROWSS && live) P.ss_part[(long)m * (2 * gridDim.y) + 2 * blockIdx.y + half] = ss;
+      }
+    }
+    if (ok && live) {
+      const float rs = P.row_scale != nullptr ? P.row_scale[m] : 1.0f;
+      (void)rs;
+      if constexpr (EPI == EPI_STORE) {
+        if (P.out_dtype == 2) {
+          const int ncols = min(BN, P.N - n0);
+#pragma unroll
+          for (int c0 = 0; c0 < Cfg::kHalf; c0 += 16) {
+            const int col = c_base + c0;
+            if (col >= ncols) break;
+            const int valid = min(16, ncols - col);
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = acc[c0 + j] * rs;
+            const long idx = (long)m * P.ld_out + n0 + col;
+            if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
+            store16(P.out, idx, P.out_dtype, v, valid);
+          }
+        }
       } else if constexpr (EPI == EPI_XPROJ_A16) {
         // columns [0,R) dt (all in half 0: R <= BN/2) | [R,R+Ns) B | [R+Ns,R+2Ns) C
         const int R = P.R, Ns = P.Ns;
