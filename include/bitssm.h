@@ -278,14 +278,15 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
  *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],
  *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]
  *   A16: r_x float [T], u bf16 [T, E], dt_low bf16 [T, R], r_dt float [T],
- *        Bm, Cm float [T, N], delta_raw float [T, E], y bf16 [T, E],
+ *        Bm, Cm float [T, N], delta float [T, E] (= softplus(delta_raw +
+ *        dt_bias), formed in the dt_proj epilogue), y bf16 [T, E],
  *        r_y float [T]
  * deq_* is the per-token factor m * r / 127 of the absmax codes; r_* the
  * RMSNorm factor. */
 typedef struct bitssm_ws_view {
   size_t q_x, deq_x, u, q_u, deq_u, Bm, Cm, q_dt, deq_dt, y, q_y, deq_y;
   size_t r_x, dt_low, r_dt, delta_raw, r_y;
-  size_t u_scale;
+  size_t u_scale, delta;
   int ld_qx, ld_qu, ld_qdt;
   int u_dtype;
 } bitssm_ws_view;

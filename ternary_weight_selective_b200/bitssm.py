@@ -69,7 +69,7 @@ class bitssm_layer(ctypes.Structure):
 class bitssm_ws_view(ctypes.Structure):
     _fields_ = [(n, _sz) for n in ("q_x", "deq_x", "u", "q_u", "deq_u", "Bm", "Cm", "q_dt",
                                    "deq_dt", "y", "q_y", "deq_y", "r_x", "dt_low", "r_dt",
-                                   "delta_raw", "r_y", "u_scale")] + \
+                                   "delta_raw", "r_y", "u_scale", "delta")] + \
                [("ld_qx", _i), ("ld_qu", _i), ("ld_qdt", _i), ("u_dtype", _i)]
 
 

@@ -128,13 +128,24 @@ int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, c
 }
 
 // W1.58A16 GEMM with exact fp32 group scales (transposed scales in P.s_t).
-template <int BN, int EPI>
-int launch_gemm_gs_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
+// Epilogue warps of the group-scaled GEMM: 8 (two column slices), or 16
+// (four slices of at least 32 columns) for a single 128-wide K group, where
+// the epilogue is the whole cost and the accumulators are few, when the two
+// pipeline stages can hold sixteen output transpose buffers.  The u^2
+// partial sums of ROWSS are laid out for 8.
+constexpr int gs_nepi(int epi, int bn, int stages) {
+  return ((epi == EPI_STORE || epi == EPI_DELTA) && stages == 2 && bn >= 128 &&
+          16 * kStageFloats * 4 <= stages * (128 * 128 + bn * 128))
+             ? 16
+             : 8;
+}
+
+template <int BN, int EPI, int kStages>
+int launch_gemm_gs_st(const void* A, long lda, const void* W, long ldw, long w_rows,
                       const GemmParams& P, cudaStream_t st) {
-  constexpr int kStage = 128 * 128 + BN * 128;
-  constexpr int kStages = (200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage);
-  using Cfg = GsConfig<BN, kStages>;
-  auto kern = ternary_gemm_gs_kernel<BN, kStages, EPI>;
+  constexpr int kNepi = gs_nepi(EPI, BN, kStages);
+  using Cfg = GsConfig<BN, kStages, kNepi>;
+  auto kern = ternary_gemm_gs_kernel<BN, kStages, EPI, kNepi>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
@@ -146,8 +157,17 @@ int launch_gemm_gs_bn(const void* A, long lda, const void* W, long ldw, long w_r
   if (!make_map(&mA, A, true, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (!make_map(&mW, W, true, P.K, w_rows, ldw, BN)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   dim3 grid((P.M + 127) / 128, (P.N + BN - 1) / BN);
-  kern<<<grid, 320, Cfg::kSmemBytes, st>>>(mA, mW, P);
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mA, mW, P);
   return launch_status();
+}
+
+// Four pipeline stages; a single 128-wide K group (dt_proj) takes two, so
+// that two CTAs (each with half of TMEM) share an SM.
+template <int BN, int EPI>
+int launch_gemm_gs_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
+                      const GemmParams& P, cudaStream_t st) {
+  if (P.K <= 128) return launch_gemm_gs_st<BN, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+  return launch_gemm_gs_st<BN, EPI, 4>(A, lda, W, ldw, w_rows, P, st);
 }
 
 // N tile of the group-scaled GEMM: whole-row epilogues need every column in
@@ -169,9 +189,12 @@ int launch_gemm_gs(const void* A, long lda, const void* W, long ldw, long w_rows
   return launch_gemm_gs_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);
 }
 
-// Partial sums of u^2 per A16 in_proj row: two per N tile (one per epilogue
-// column half).
-inline int rowss_parts(int E) { return 2 * ((E + gs_bn(E, false) - 1) / gs_bn(E, false)); }
+// Partial sums of u^2 per A16 in_proj row: one per N tile and epilogue
+// column slice.
+inline int rowss_parts(int E) {
+  const int bn = gs_bn(E, false);
+  return (gs_nepi(EPI_ROWSS, bn, 4) / 4) * ((E + bn - 1) / bn);
+}
 
 // Transposed fp32 group scales of an expanded bf16 matrix: [G][ld_s]
 inline int scale_groups(int k_in) { return (k_in + 127) / 128; }
@@ -244,12 +267,12 @@ int launch_expand(const ExpandJobs& jobs, bool bf16, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------ scan launch
-template <int NPT, bool FUSED, int RV, typename Tu, typename Td, typename Ty>
+template <int NPT, bool FUSED, int RV, typename Tu, typename Td, typename Ty, bool DFIN>
 int launch_scan_t(const ScanParams& P, cudaStream_t st) {
   constexpr int TPC = kScanN / NPT;
   constexpr int CE = 128 / TPC;
   constexpr int smem = 2 * ScanStage<CE, FUSED, Tu, Td>::kBytes;
-  auto kern = selective_scan_kernel<NPT, FUSED, RV, Tu, Td, Ty>;
+  auto kern = selective_scan_kernel<NPT, FUSED, RV, Tu, Td, Ty, DFIN>;
   static bool attr_set = false;
   if (!attr_set && smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -274,29 +297,37 @@ int scan_npt_override() {
   return v;
 }
 
-template <bool FUSED, int RV, typename Tu, typename Td, typename Ty>
+template <bool FUSED, int RV, typename Tu, typename Td, typename Ty, bool DFIN>
 int launch_scan_rv(const ScanParams& P, cudaStream_t st) {
   const long channels = (long)P.B * P.E;
   const long want = (long)num_sms() * 4 * 48;
   int npt = channels >= want ? 16 : (channels * 2 >= want ? 8 : 4);
+  if (DFIN) {
+    // with delta read ready-made, the per-step work is the recurrence alone:
+    // take the most states per thread that still gives ~3 warps per SM
+    // sub-partition (measured: 4 states per thread at B*E = 16384)
+    const long threads_min = (long)num_sms() * 4 * 3 * 32;
+    npt = channels * 2 >= threads_min ? 8 : 4;
+    if (channels >= threads_min) npt = 16;
+  }
   if (scan_npt_override() != 0) npt = scan_npt_override();
-  if (npt == 16) return launch_scan_t<16, FUSED, RV, Tu, Td, Ty>(P, st);
-  if (npt == 8) return launch_scan_t<8, FUSED, RV, Tu, Td, Ty>(P, st);
-  return launch_scan_t<4, FUSED, RV, Tu, Td, Ty>(P, st);
+  if (npt == 16) return launch_scan_t<16, FUSED, RV, Tu, Td, Ty, DFIN>(P, st);
+  if (npt == 8) return launch_scan_t<8, FUSED, RV, Tu, Td, Ty, DFIN>(P, st);
+  return launch_scan_t<4, FUSED, RV, Tu, Td, Ty, DFIN>(P, st);
 }
 
-template <bool FUSED, typename Tu, typename Td, typename Ty>
+template <bool FUSED, typename Tu, typename Td, typename Ty, bool DFIN = false>
 int launch_scan(const ScanParams& P, cudaStream_t st) {
   if (std::is_same<Tu, int16_t>::value != (P.u_scale != nullptr)) return BITSSM_ERR_INVALID_ARG;
   if constexpr (FUSED) {
     switch (P.R / 16) {  // Delta-up width (dt_rank padded to 16)
-      case 1: return launch_scan_rv<true, 1, Tu, Td, Ty>(P, st);
-      case 2: return launch_scan_rv<true, 2, Tu, Td, Ty>(P, st);
-      case 3: case 4: return launch_scan_rv<true, 4, Tu, Td, Ty>(P, st);
-      default: return launch_scan_rv<true, 8, Tu, Td, Ty>(P, st);
+      case 1: return launch_scan_rv<true, 1, Tu, Td, Ty, false>(P, st);
+      case 2: return launch_scan_rv<true, 2, Tu, Td, Ty, false>(P, st);
+      case 3: case 4: return launch_scan_rv<true, 4, Tu, Td, Ty, false>(P, st);
+      default: return launch_scan_rv<true, 8, Tu, Td, Ty, false>(P, st);
     }
   }
-  return launch_scan_rv<false, 1, Tu, Td, Ty>(P, st);
+  return launch_scan_rv<false, 1, Tu, Td, Ty, DFIN>(P, st);
 }
 
 // ------------------------------------------------------------ validation
@@ -389,7 +420,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   bitssm_ws_view& v = P.v;
   v.q_x = v.deq_x = v.u = v.q_u = v.deq_u = v.Bm = v.Cm = v.q_dt = v.deq_dt = v.y = v.q_y = v.deq_y = none;
   v.r_x = v.dt_low = v.r_dt = v.delta_raw = v.r_y = none;
-  v.u_scale = none;
+  v.u_scale = v.delta = none;
   v.u_dtype = P.a16 ? BITSSM_BF16 : BITSSM_F32;
   P.ss_u = none;
   auto take = [&](size_t bytes) {
@@ -423,7 +454,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
     v.r_dt = take(T * 4);
     v.Bm = take(T * P.N * 4);
     v.Cm = take(T * P.N * 4);
-    v.delta_raw = take(T * P.E * 4);
+    v.delta = take(T * P.E * 4);
     v.y = take(T * P.E * 2);
     v.r_y = take(T * 4);
   }
@@ -739,15 +770,16 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     if (rc) return rc;
   }
   mk.mark();
-  {  // dt_proj: delta_raw = r_dt * acc (f32)
+  {  // dt_proj: delta = softplus(r_dt * acc + dt_bias) (f32)
     GemmParams G;
     std::memset(&G, 0, sizeof(G));
     G.M = T; G.N = P.E; G.K = P.R;
     G.out_dtype = BITSSM_F32;
     G.row_scale = at<float>(ws, v.r_dt);
-    G.out = at<float>(ws, v.delta_raw); G.ld_out = P.E;
+    G.bias = p->dt_bias;
+    G.out = at<float>(ws, v.delta); G.ld_out = P.E;
     G.s_t = reinterpret_cast<const float*>(wexp + P.s_up); G.ld_s = scale_ld(P.E);
-    rc = launch_gemm_gs<EPI_STORE>(at<__nv_bfloat16>(ws, v.dt_low), P.ld_R, wexp + P.w_up, P.ld_R,
+    rc = launch_gemm_gs<EPI_DELTA>(at<__nv_bfloat16>(ws, v.dt_low), P.ld_R, wexp + P.w_up, P.ld_R,
                                    P.E, G, st);
     if (rc) return rc;
   }
@@ -756,12 +788,12 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     ScanParams S;
     std::memset(&S, 0, sizeof(S));
     S.u = at<__nv_bfloat16>(ws, v.u);
-    S.delta_raw = at<float>(ws, v.delta_raw);
+    S.delta_raw = at<float>(ws, v.delta);  // already delta (bias and softplus applied)
     S.bias = p->dt_bias; S.A = p->A; S.D = p->D;
     S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
     S.y = at<__nv_bfloat16>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
-    rc = launch_scan<false, __nv_bfloat16, float, __nv_bfloat16>(S, st);
+    rc = launch_scan<false, __nv_bfloat16, float, __nv_bfloat16, true>(S, st);
     if (rc) return rc;
   }
   mk.mark();

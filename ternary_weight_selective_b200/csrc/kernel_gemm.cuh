@@ -32,6 +32,7 @@ enum EpiKind : int {
   EPI_XPROJ_A8 = 2,   // A8 x_proj: dt codes + deq_dt from the int32 row, B and C (f32)
   EPI_ROWSS = 3,      // A16 in_proj: u (bf16) = acc * r_x + partial sum(u^2) per tile
   EPI_XPROJ_A16 = 4,  // A16 x_proj: dt_low (bf16) + r_dt, B and C (f32)
+  EPI_DELTA = 5,      // A16 dt_proj: delta = softplus(acc * row_scale[m] + bias[n]) -> f32
 };
 
 struct GemmParams {
@@ -59,6 +60,7 @@ struct GemmParams {
   int ss_nparts;
   int ss_count;                // number of columns the partial sums cover
   float* r_out;                // EPI_XPROJ_A16: r_dt [M]
+  const float* bias;           // EPI_DELTA: [N]
   // group-scaled (W1.58A16) kernel: fp32 scales transposed, s_t[g * ld_s + n]
   const float* s_t;
   long ld_s;
@@ -547,7 +549,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int NEPI = 8>
 struct GsConfig {
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytes = BN * 128;
@@ -561,16 +563,22 @@ struct GsConfig {
   static constexpr int kScaleOffset = STAGES * kStageBytes;
   static constexpr int kBarOffset = kScaleOffset + kScaleSlots * BN * 4;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
-  static constexpr int kHalf = BN / 2;  // columns per epilogue warp
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
-  static_assert(8 * kStageFloats * 4 <= STAGES * kStageBytes, "output staging");
+  // NEPI epilogue warps: NEPI/4 per TMEM lane quadrant, each owning a
+  // column slice of kHalf columns
+  static constexpr int kSlices = NEPI / 4;
+  static constexpr int kHalf = BN / kSlices;  // columns per epilogue warp
+  static constexpr int kThreads = 64 + 32 * NEPI;
+  static_assert(NEPI == 8 || NEPI == 16, "NEPI");
+  static_assert(BN % (32 * kSlices) == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(NEPI * kStageFloats * 4 <= STAGES * kStageBytes, "output staging");
 };
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(320, 1)
+template <int BN, int STAGES, int EPI, int NEPI>
+__global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
     ternary_gemm_gs_kernel(const __grid_constant__ CUtensorMap mapA,
                            const __grid_constant__ CUtensorMap mapW, GemmParams P) {
-  using Cfg = GsConfig<BN, STAGES>;
+  using Cfg = GsConfig<BN, STAGES, NEPI>;
+  static_assert(EPI != EPI_XPROJ_A16 || NEPI == 8, "the x_proj epilogue keeps dt in slice 0");
   constexpr int kPanel = 64;             // bf16 elements per 128-byte panel
   constexpr int kPanelsPerGroup = 2;     // 128-element weight groups
   extern __shared__ uint8_t smem_raw[];
@@ -590,6 +598,9 @@ __global__ void __launch_bounds__(320, 1)
   const int n0 = blockIdx.y * BN;
   const int num_panels = (P.K + kPanel - 1) / kPanel;
   const int num_groups = (num_panels + kPanelsPerGroup - 1) / kPanelsPerGroup;
+  // one 256-column accumulator buffer per group in flight: a single group
+  // needs one, leaving the other half of TMEM to a second CTA on the SM
+  const uint32_t tmem_cols = num_groups > 1 ? 512u : 256u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -598,14 +609,14 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull_bar(b), 1);
-      mbar_init(pempty_bar(b), 8);
+      mbar_init(pempty_bar(b), NEPI);
     }
     fence_mbar_init();
     tma_prefetch_desc(&mapA);
     tma_prefetch_desc(&mapW);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -663,7 +674,7 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp >= 2) {
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - 2) >> 2;  // column slice
     const int row = q * 32 + lane;
     const int m = m0 + row;
     const bool live = m < P.M;
@@ -681,9 +692,9 @@ __global__ void __launch_bounds__(320, 1)
       // the group's scale row landed with its first panel, before the MMAs
       const float4* s4 = reinterpret_cast<const float4*>(
           smem + Cfg::kScaleOffset + (g % Cfg::kScaleSlots) * (BN * 4) + c_base * 4);
-      // columns per TMEM round trip: 16 with 128 accumulators per thread
-      // (register budget), else 32
-      constexpr int kLd = Cfg::kHalf >= 128 ? 16 : 32;
+      // columns per TMEM round trip: 16, or 32 for a 32-column slice
+      // (register budget of the accumulators)
+      constexpr int kLd = Cfg::kHalf == 32 ? 32 : 16;
 #pragma unroll
       for (int c0 = 0; c0 < Cfg::kHalf; c0 += kLd) {
         uint32_t r[kLd];
@@ -707,8 +718,8 @@ __global__ void __launch_bounds__(320, 1)
     // STORE / ROWSS with a float or bf16 output: coalesced stores through a
     // per-warp transpose buffer in the (now idle) pipeline stages.  Every
     // lane takes part (rows >= M are skipped inside the store).
-    if constexpr (EPI == EPI_STORE || EPI == EPI_ROWSS) {
-      const int odt = EPI == EPI_ROWSS ? 1 : P.out_dtype;
+    if constexpr (EPI == EPI_STORE || EPI == EPI_ROWSS || EPI == EPI_DELTA) {
+      const int odt = EPI == EPI_ROWSS ? 1 : EPI == EPI_DELTA ? 0 : P.out_dtype;
       if (ok && odt != 2) {
         const float rs = (live && P.row_scale != nullptr) ? P.row_scale[m] : 1.0f;
         float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * kStageFloats;
@@ -723,12 +734,19 @@ __global__ void __launch_bounds__(320, 1)
             v[j] = acc[c0 + j] * rs;
             if (EPI == EPI_ROWSS && c_base + c0 + j < ncols) ss = fmaf(v[j], v[j], ss);
           }
+          if constexpr (EPI == EPI_DELTA) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int col = c_base + c0 + j;
+              v[j] = softplus_fast(v[j] + (col < ncols ? __ldg(P.bias + n0 + col) : 0.f));
+            }
+          }
           if (odt == 1)
             warp_store_block<1>(stg, v, lane, P.out, res, P.ld_out, m0 + q * 32, n0 + c_base + c0, P.M, P.N);
           else
             warp_store_block<0>(stg, v, lane, P.out, res, P.ld_out, m0 + q * 32, n0 + c_base + c0, P.M, P.N);
         }
-        if (EPI == EPI_ROWSS && live) P.ss_part[(long)m * (2 * gridDim.y) + 2 * blockIdx.y + half] = ss;
+        if (EPI == EPI_ROWSS && live) P.ss_part[(long)m * (Cfg::kSlices * gridDim.y) + Cfg::kSlices * blockIdx.y + half] = ss;
       }
     }
     if (ok && live) {
@@ -781,7 +799,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, tmem_cols);
   }
 }
 

@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace bitssm {
 
 constexpr float kEpsNorm = 1e-5f;
@@ -57,8 +59,28 @@ __device__ __forceinline__ int quant_code(float v, float sigma) {
 // valued or real x lands in [2^23, 2^24), where the IEEE round-to-nearest-
 // even addition performs rint(x) and the low mantissa bits hold rint(x) in
 // two's complement.
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
+
+// softplus(z) = max(z, 0) + log1p(t), t = exp(-|z|) in (0, 1], with log1p(t)
+// = t * p(t) and p a degree-8 least-squares fit of log1p(t)/t on [0, 1]
+// (coefficients from gen_softplus_poly.py; relative error ~3e-8 before
+// float32 rounding).  One exp2 and nine FMAs.
+__device__ __forceinline__ float softplus_fast(float z) {
+  const float t = ex2_approx(-fabsf(z) * kLog2e);
+  float p = 5.253457797e-03f;
+  p = fmaf(p, t, -2.958850739e-02f);
+  p = fmaf(p, t, 7.836166802e-02f);
+  p = fmaf(p, t, -1.367476971e-01f);
+  p = fmaf(p, t, 1.911143108e-01f);
+  p = fmaf(p, t, -2.484436989e-01f);
+  p = fmaf(p, t, 3.331927134e-01f);
+  p = fmaf(p, t, -4.999950152e-01f);
+  p = fmaf(p, t, 9.999999705e-01f);
+  return fmaxf(z, 0.f) + t * p;
+}
+
 __device__ __forceinline__ float i2f_exact(int a) { return __int_as_float(a + kMagicBits) - kMagic; }
 // Bit pattern whose low byte is the int8 code rint(v * sigma).  With
 // sigma = 127 / max|v| the product never exceeds 127 in magnitude (so the
