@@ -307,6 +307,13 @@ int launch_scan_rv(const ScanParams& P, cudaStream_t st) {
     // take the most states per thread that still gives ~3 warps per SM
     // sub-partition (measured: 4 states per thread at B*E = 16384)
     const long threads_min = (long)num_sms() * 4 * 3 * 32;
+    npt = channels >= threads_min ? 16 : (channels * 2 >= threads_min ? 8 : 4);
+  }
+  if (DFIN) {
+    // with delta read ready-made, the per-step work is the recurrence alone:
+    // take the most states per thread that still gives ~3 warps per SM
+    // sub-partition (measured: 4 states per thread at B*E = 16384)
+    const long threads_min = (long)num_sms() * 4 * 3 * 32;
     npt = channels * 2 >= threads_min ? 8 : 4;
     if (channels >= threads_min) npt = 16;
   }
