@@ -180,6 +180,10 @@ def run_ours(args):
     out = torch.empty_like(xd)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     n_layers = len(dl)
+    # decode workloads: every step is one bitssm_step (one token per sequence)
+    # with the recurrent state carried in h_state
+    decode = args.workload.endswith("_decode")
+    h_state = torch.zeros((B, wl.d_inner, wl.d_state), dtype=torch.float32, device="cuda")
 
     def new_events(n):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -208,7 +212,10 @@ def run_ours(args):
             h_in = xd
             for li, d_l in enumerate(dl):
                 res = h_in if n_layers > 1 else None
-                if evs is None:
+                if evs is None and decode:
+                    abi.bitssm_step(d_l.layer, h_in, out, res, h_state, B, dtype, act, ws.addr,
+                                    nbytes, st)
+                elif evs is None:
                     abi.bitssm_forward(d_l.layer, h_in, out, res, B, L, dtype, act, ws.addr,
                                        nbytes, st)
                 else:
@@ -328,8 +335,12 @@ def run_ours(args):
         x_dev2.copy_(x_host, non_blocking=True)
         h_in = x_dev2
         for d_l in dl:
-            abi.bitssm_forward(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B, L, dtype,
-                               act, ws.addr, nbytes, torch.cuda.current_stream())
+            if decode:
+                abi.bitssm_step(d_l.layer, h_in, out, h_in if n_layers > 1 else None, h_state, B,
+                                dtype, act, ws.addr, nbytes, torch.cuda.current_stream())
+            else:
+                abi.bitssm_forward(d_l.layer, h_in, out, h_in if n_layers > 1 else None, B, L,
+                                   dtype, act, ws.addr, nbytes, torch.cuda.current_stream())
             h_in = out
         out_host.copy_(out, non_blocking=True)
 
@@ -414,6 +425,8 @@ def run_ours(args):
                    "d_inner": wl.d_inner, "d_state": wl.d_state, "dt_rank": wl.dt_rank,
                    "layers": n_layers, "io_dtype": wl.io_dtype, "act_mode": wl.act_mode,
                    "parallelism": f"replica x{world}" if world > 1 else "single",
+                   "mode": "decode: bitssm_step, one token per sequence, state carried"
+                           if decode else "forward over whole sequences",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)"},
         "roofline": roof,
         "kernel_share": share,

@@ -248,6 +248,25 @@ int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const 
                          int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
                          void* const* events, int n_events, void* stream);
 
+/* ---------------------------------------------------------------------
+ * Forward with a carried state: the recurrent form of the same layer
+ * ("Ternary Mamba" abstract: SSMs offer linear-time inference; the state h
+ * is all that links one step to the next).  h [B, d_inner, d_state] float:
+ * the scan starts from h (instead of zero) and h is overwritten with the
+ * state after the last step.  Every other stage is token-local, so running
+ * a sequence in pieces (or one token at a time) with the same h gives the
+ * results of one call over the whole sequence.  Arguments otherwise as
+ * bitssm_forward (same workspace size for the same B and L); h must not
+ * alias x, out or the workspace.  Errors as bitssm_forward; a NULL h is
+ * BITSSM_ERR_INVALID_ARG.
+ * bitssm_step is the decode step: L = 1, x and out [B, d_model].
+ * --------------------------------------------------------------------- */
+int bitssm_forward_state(const bitssm_layer* p, const void* x, void* out, const void* residual,
+                         float* h, int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* stream);
+int bitssm_step(const bitssm_layer* p, const void* x, void* out, const void* residual, float* h,
+                int B, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream);
+
 /* Residual stack (TriSSM README Overview table: 12 layers at d = 256):
  * out = x; for each layer l: out = out + mixer_l(out), rounded to `dtype`.
  * `layers` is a host array of n_layers layer structs of identical shapes.

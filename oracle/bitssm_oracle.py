@@ -325,8 +325,11 @@ class TernaryLayer:
         self.N = lw.W_B.shape[0]
 
 
-def bitssm_layer_a8(x: np.ndarray, P: TernaryLayer) -> tuple[np.ndarray, dict]:
+def bitssm_layer_a8(x: np.ndarray, P: TernaryLayer, h0=None) -> tuple[np.ndarray, dict]:
     """One BitSSM mixer with int8 activations, x [B, L, d_model] -> out.
+    h0 [B, d_inner, N] (None = zero) is the scan's starting state; the
+    state after the last step is returned as stages["h_last"] (the recurrent
+    form: [TernaryMamba] abstract, linear-time inference).
 
     Readings: in_proj and out_proj are ternary BitLinears too; the Delta path
     is low rank (d_inner -> dt_rank -> d_inner), both factors ternary;
@@ -357,20 +360,21 @@ def bitssm_layer_a8(x: np.ndarray, P: TernaryLayer) -> tuple[np.ndarray, dict]:
                                               P.s["W_dt_up"])
     delta = softplus(delta_raw + P.dt_bias[None])
     E = u.shape[1]
-    y, _ = selective_scan(u.reshape(Bsz, L, E), delta.reshape(Bsz, L, E), P.A,
-                          Bm.reshape(Bsz, L, N), Cm.reshape(Bsz, L, N), P.D)
+    y, h_last = selective_scan(u.reshape(Bsz, L, E), delta.reshape(Bsz, L, E), P.A,
+                               Bm.reshape(Bsz, L, N), Cm.reshape(Bsz, L, N), P.D, h0)
     out, st_out = bitlinear_a8(y.reshape(T, E), P.Wq["W_out"], P.s["W_out"])
     stages = dict(q_x=st_in["q"], deq_x=st_in["deq"], acc_in=st_in["acc"], u=u,
                   q_u=st_x["q"], deq_u=deq_u, acc_x=acc_x, Bm=Bm, Cm=Cm, dt_low=dt_low,
                   q_dt=st_dt["q"], deq_dt=st_dt["deq"], delta_raw=delta_raw, delta=delta,
                   y=y.reshape(T, E), q_y=st_out["q"], deq_y=st_out["deq"],
-                  acc_out=st_out["acc"])
+                  acc_out=st_out["acc"], h_last=h_last)
     return out.reshape(Bsz, L, -1), stages
 
 
-def bitssm_layer_a16(x: np.ndarray, P: TernaryLayer) -> tuple[np.ndarray, dict]:
+def bitssm_layer_a16(x: np.ndarray, P: TernaryLayer, h0=None) -> tuple[np.ndarray, dict]:
     """One BitSSM mixer in W1.58A16 form ([TernaryMamba] abstract): every
-    projection is ``bitlinear_a16`` on the 16-bit activation row before it."""
+    projection is ``bitlinear_a16`` on the 16-bit activation row before it.
+    h0 / stages["h_last"]: the carried state, as in ``bitssm_layer_a8``."""
     Bsz, L, d = x.shape
     T = Bsz * L
     g = P.group
@@ -383,18 +387,26 @@ def bitssm_layer_a16(x: np.ndarray, P: TernaryLayer) -> tuple[np.ndarray, dict]:
     delta_raw = bitlinear_a16(dt_low, P.Wq["W_dt_up"], P.s["W_dt_up"], g)
     delta = softplus(delta_raw + P.dt_bias[None])
     E = u.shape[1]
-    y, _ = selective_scan(u.reshape(Bsz, L, E), delta.reshape(Bsz, L, E), P.A,
-                          Bm.reshape(Bsz, L, N), Cm.reshape(Bsz, L, N), P.D)
+    y, h_last = selective_scan(u.reshape(Bsz, L, E), delta.reshape(Bsz, L, E), P.A,
+                               Bm.reshape(Bsz, L, N), Cm.reshape(Bsz, L, N), P.D, h0)
     out = bitlinear_a16(y.reshape(T, E), P.Wq["W_out"], P.s["W_out"], g)
     stages = dict(u=u, dt_low=dt_low, Bm=Bm, Cm=Cm, delta_raw=delta_raw, delta=delta,
-                  y=y.reshape(T, E))
+                  y=y.reshape(T, E), h_last=h_last)
     return out.reshape(Bsz, L, -1), stages
 
 
-def bitssm_layer(x, P: TernaryLayer):
+def bitssm_layer(x, P: TernaryLayer, h0=None):
     if P.act_mode == "A16":
-        return bitssm_layer_a16(x, P)
-    return bitssm_layer_a8(x, P)
+        return bitssm_layer_a16(x, P, h0)
+    return bitssm_layer_a8(x, P, h0)
+
+
+def bitssm_step(x_t: np.ndarray, P: TernaryLayer, h: np.ndarray):
+    """The decode step: one token per sequence, x_t [B, d_model], state h
+    [B, d_inner, N] -> (out [B, d_model], new h).  The same layer with L = 1
+    and the state carried (the recurrence is the only link between steps)."""
+    out, st = bitssm_layer(np.asarray(x_t)[:, None, :], P, h)
+    return out[:, 0, :], st["h_last"]
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:

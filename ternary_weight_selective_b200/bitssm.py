@@ -90,6 +90,8 @@ _SIGS = {
                                     _i, _i, _i, _i, _i, _vp]),
     "bitssm_workspace_size": (_i, [_P_LAYER, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "bitssm_forward": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "bitssm_forward_state": (_i, [_P_LAYER, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "bitssm_step": (_i, [_P_LAYER, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "bitssm_stack_forward": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "bitssm_forward_launches": (_i, [_P_LAYER, _i]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
@@ -205,6 +207,21 @@ def bitssm_forward(layer: bitssm_layer, x, out, residual, B, L, dtype, act_mode,
     _check(_lib.bitssm_forward(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual), B, L,
                                dtype, act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitssm_forward")
+
+
+def bitssm_forward_state(layer: bitssm_layer, x, out, residual, h, B, L, dtype, act_mode, ws,
+                         ws_bytes, stream=None):
+    _check(_lib.bitssm_forward_state(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual),
+                                     _ptr(h), B, L, dtype, act_mode, _ptr(ws), ws_bytes,
+                                     _stream(stream)),
+           "bitssm_forward_state")
+
+
+def bitssm_step(layer: bitssm_layer, x, out, residual, h, B, dtype, act_mode, ws, ws_bytes,
+                stream=None):
+    _check(_lib.bitssm_step(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual), _ptr(h), B,
+                            dtype, act_mode, _ptr(ws), ws_bytes, _stream(stream)),
+           "bitssm_step")
 
 
 def bitssm_forward_launches(layer: bitssm_layer, act_mode) -> int:

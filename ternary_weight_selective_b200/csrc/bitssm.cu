@@ -602,7 +602,7 @@ int launch_post(const PostParams& Q, const void* w, long ldw, cudaStream_t st) {
 
 int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp,
                      const void* x, void* out, const void* residual, int B, int L, int dtype,
-                     void* ws, cudaStream_t st, Marks& mk) {
+                     void* ws, cudaStream_t st, Marks& mk, float* h) {
   const bitssm_ws_view& v = P.v;
   const bool keep = (p->flags & BITSSM_KEEP_CODES) != 0;
   int rc;
@@ -640,6 +640,7 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
     S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
     S.y = at<float>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
+    S.h0 = h; S.h_last = h;  // carried state (nullable): read, then overwritten
     rc = launch_scan<true, int16_t, float, float>(S, st);
     if (rc) return rc;
   }
@@ -662,7 +663,7 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
 
 int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, const void* x,
                void* out, const void* residual, int B, int L, int dtype, void* ws,
-               cudaStream_t st, Marks& mk) {
+               cudaStream_t st, Marks& mk, float* h) {
   const bitssm_ws_view& v = P.v;
   const int T = P.T;
   int rc;
@@ -714,6 +715,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
     S.y = at<float>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
+    S.h0 = h; S.h_last = h;  // carried state (nullable): read, then overwritten
     rc = launch_scan<true, float, float, float>(S, st);
     if (rc) return rc;
   }
@@ -742,7 +744,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
 
 int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, const void* x,
                 void* out, const void* residual, int B, int L, void* ws, cudaStream_t st,
-                Marks& mk) {
+                Marks& mk, float* h) {
   const bitssm_ws_view& v = P.v;
   const int T = P.T;
   int rc;
@@ -800,6 +802,7 @@ int forward_a16(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, 
     S.Bm = at<float>(ws, v.Bm); S.Cm = at<float>(ws, v.Cm);
     S.y = at<__nv_bfloat16>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
+    S.h0 = h; S.h_last = h;  // carried state (nullable): read, then overwritten
     rc = launch_scan<false, __nv_bfloat16, float, __nv_bfloat16, true>(S, st);
     if (rc) return rc;
   }
@@ -1075,7 +1078,7 @@ namespace bitssm {
 namespace {
 int forward_impl(const bitssm_layer* p, const void* x, void* out, const void* residual, int B,
                  int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream,
-                 Marks& mk) {
+                 Marks& mk, float* h = nullptr) {
   int rc = check_layer_args(p, B, L, dtype, act_mode);
   if (rc) return rc;
   const long T = (long)B * L;
@@ -1098,10 +1101,10 @@ int forward_impl(const bitssm_layer* p, const void* x, void* out, const void* re
     wexp = reinterpret_cast<const uint8_t*>(ws);
   }
   if (act_mode == BITSSM_A8)
-    rc = a8_fused(P) ? forward_a8_fused(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk)
-                     : forward_a8(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk);
+    rc = a8_fused(P) ? forward_a8_fused(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk, h)
+                     : forward_a8(p, P, wexp, x, out, residual, B, L, dtype, ws, st, mk, h);
   else
-    rc = forward_a16(p, P, wexp, x, out, residual, B, L, ws, st, mk);
+    rc = forward_a16(p, P, wexp, x, out, residual, B, L, ws, st, mk, h);
   if (rc == BITSSM_OK && mk.failed) rc = BITSSM_ERR_CUDA;
   return rc;
 }
@@ -1114,6 +1117,19 @@ int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* 
                    int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream) {
   Marks mk;
   return forward_impl(p, x, out, residual, B, L, dtype, act_mode, ws, ws_bytes, stream, mk);
+}
+
+int bitssm_forward_state(const bitssm_layer* p, const void* x, void* out, const void* residual,
+                         float* h, int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (h == nullptr) return BITSSM_ERR_INVALID_ARG;
+  Marks mk;
+  return forward_impl(p, x, out, residual, B, L, dtype, act_mode, ws, ws_bytes, stream, mk, h);
+}
+
+int bitssm_step(const bitssm_layer* p, const void* x, void* out, const void* residual, float* h,
+                int B, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream) {
+  return bitssm_forward_state(p, x, out, residual, h, B, 1, dtype, act_mode, ws, ws_bytes, stream);
 }
 
 int bitssm_forward_launches(const bitssm_layer* p, int act_mode) {

@@ -69,6 +69,8 @@ WORKLOADS = {
     "stack12": Workload("stack12", 64, 256, 256, 512, 16, 16, "bf16", "A8", layers=12, source="embed"),
     "mamba2_1p3b_a16": Workload("mamba2_1p3b_a16", 4, 2048, 2048, 4096, 16, 128, "bf16", "A16"),
     "long16k": Workload("long16k", 16, 16384, 256, 512, 16, 16, "bf16", "A8", source="embed"),
+    # decode: one token for each of 64 sequences, the state carried in h
+    "trissm_decode": Workload("trissm_decode", 64, 1, 256, 512, 16, 16, "bf16", "A8"),
 }
 
 
