@@ -132,23 +132,45 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- byte counts
 
-def scan_bytes_per_token(E, N, R_pad):
-    """Algorithmic bytes of the fused scan kernel per token: read u (fp32),
-    the Delta-down codes and their factor, B and C (fp32); write y (fp32)."""
-    return E * 4 + R_pad + 4 + 2 * N * 4 + E * 4
+def scan_bytes_per_token(E, N, R_pad, a16=False):
+    """Algorithmic HBM bytes of the scan kernel per token.
+    A8 (Delta-up fused): read u (int16 accumulators + one fp32 scale), the
+    Delta-down codes and their factor, B and C (fp32); write y (fp32).
+    A16: read u (bf16), delta (fp32), B and C; write y (bf16)."""
+    if a16:
+        return E * 2 + E * 4 + 2 * N * 4 + E * 2
+    return E * 2 + 4 + R_pad + 4 + 2 * N * 4 + E * 4
 
 
-def layer_bytes_per_token(wl):
-    """Algorithmic HBM bytes per token of the fused A8 forward: the pre kernel
-    reads x and writes u (fp32), B, C, the dt codes and their factor; the scan
-    reads those and writes y (fp32); the post kernel reads y and writes out."""
+def pre_bytes_per_token(wl):
+    """bitssm_pre_kernel: read x; write u (int16 + scale), B, C, dt codes + factor."""
     d, E, N = wl.d_model, wl.d_inner, wl.d_state
     Rp = (wl.dt_rank + 15) // 16 * 16
     io = 2 if wl.io_dtype == "bf16" else 4
-    pre = d * io + E * 4 + 2 * N * 4 + Rp + 4
-    scan = scan_bytes_per_token(E, N, Rp)
-    post = E * 4 + d * io
-    return pre + scan + post
+    return d * io + E * 2 + 4 + 2 * N * 4 + Rp + 4
+
+
+def post_bytes_per_token(wl):
+    """bitssm_post_kernel: read y (fp32); write out."""
+    io = 2 if wl.io_dtype == "bf16" else 4
+    return wl.d_inner * 4 + wl.d_model * io
+
+
+def layer_bytes_per_token(wl):
+    """Algorithmic HBM bytes per token of one forward (activations only; the
+    weights are read once per call and do not scale with tokens)."""
+    d, E, N = wl.d_model, wl.d_inner, wl.d_state
+    Rp = (wl.dt_rank + 15) // 16 * 16
+    if wl.act_mode == "A16":
+        R = wl.dt_rank
+        rms_x = d * 2
+        in_proj = d * 2 + E * 2
+        x_proj = E * 2 + R * 2 + 2 * N * 4 + 4
+        dt_proj = R * 2 + E * 4
+        rms_y = E * 2
+        out_proj = E * 2 + d * 2
+        return rms_x + in_proj + x_proj + dt_proj + scan_bytes_per_token(E, N, Rp, True) + rms_y + out_proj
+    return pre_bytes_per_token(wl) + scan_bytes_per_token(E, N, Rp) + post_bytes_per_token(wl)
 
 
 # ---------------------------------------------------------------- our arm
@@ -396,7 +418,7 @@ def run_ours(args):
         t_s = avg_kernel_ms[dom] / 1e3
         achieved = exps / t_s / 1e12
         peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e12
-        hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp)
+        hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp, act == abi.A16)
         roof = {"kernel": names[dom], "bound": "alu", "unit": "Tex2/s",
                 "achieved": round(achieved, 4), "peak": round(peak, 4),
                 "frac": round(achieved / peak, 4),
@@ -408,11 +430,23 @@ def run_ours(args):
                 "hbm_frac": round(hbm_bytes / t_s / 1e9 / peaks["hbm_gbs"], 4),
                 "hbm_peak_source": f"{peak_kind} hbm_gbs"}
     else:
+        # the fused pre or post kernel: its own activation bytes plus its
+        # prepared int8 weights (read once per launch)
         t_s = avg_kernel_ms[dom] / 1e3
-        bytes_all = T * layer_bytes_per_token(wl)
+        d, E = wl.d_model, wl.d_inner
+        r16 = lambda v: (v + 15) // 16 * 16
+        if names[dom].startswith("bitssm_pre"):
+            kbytes = T * pre_bytes_per_token(wl) + E * r16(d) + 64 * r16(E)
+        elif names[dom].startswith("bitssm_post"):
+            kbytes = T * post_bytes_per_token(wl) + d * r16(E)
+        else:
+            kbytes = None
+        ach = None if kbytes is None else kbytes / t_s / 1e9
         roof = {"kernel": names[dom], "bound": "hbm", "unit": "GB/s",
-                "achieved": round(bytes_all / t_s / 1e9, 1), "peak": peaks["hbm_gbs"],
-                "frac": None, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs"}
+                "achieved": None if ach is None else round(ach, 1), "peak": peaks["hbm_gbs"],
+                "frac": None if ach is None else round(ach / peaks["hbm_gbs"], 4),
+                "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
+                "bytes_per_launch": kbytes}
     layer_gbs = T * layer_bytes_per_token(wl) / (ms_per_step / n_layers / 1e3) / 1e9
 
     line = {
