@@ -275,6 +275,34 @@ int bitssm_stack_forward(const bitssm_layer* layers, int n_layers, const void* x
                          int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* ---------------------------------------------------------------------
+ * The forward on host buffers, copies overlapped with the computation.
+ * n_layers == 1: out = mixer(x) as bitssm_forward (no residual);
+ * n_layers > 1: the residual stack as bitssm_stack_forward.
+ * x_host, out_host: [B, L, d_model] of `dtype` in host memory (page-locked,
+ * e.g. cudaHostAlloc, for the copies to overlap; pageable memory gives the
+ * same results, serialised).  x_dev, out_dev: caller-owned device buffers of
+ * the same size (the copies' staging; out_dev also holds the result).
+ * The batch is cut into n_chunks (1..16) groups of whole sequences; chunk
+ * i's host-to-device copy, forward and device-to-host copy run on a helper
+ * stream, `stream` and a second helper stream, ordered by events, so copies
+ * of neighbouring chunks overlap the forward (sequences are independent, so
+ * the result equals one call over the whole batch).  ws: bitssm_workspace_size
+ * for one chunk (ceil(B / n_chunks) sequences) is enough.  Everything queued
+ * on `stream` before the call happens first; the work of the call is
+ * complete when `stream` reaches the point after it.  The two helper streams
+ * and their events are created on the first call on each device and kept;
+ * calls from several host threads are serialised inside.  Weights should be
+ * prepared (bitssm_prepare_weights): otherwise every chunk expands them.
+ * Errors: BITSSM_ERR_INVALID_ARG (NULL buffers, n_chunks out of range,
+ * dtype), the errors of bitssm_forward, BITSSM_ERR_CUDA for a failed copy or
+ * stream operation (bitssm_last_error has the message).  The pages give no
+ * interface for this; it is the host-facing form of the same forward.
+ * --------------------------------------------------------------------- */
+int bitssm_forward_host(const bitssm_layer* layers, int n_layers, const void* x_host,
+                        void* out_host, int B, int L, int dtype, int act_mode, void* x_dev,
+                        void* out_dev, void* ws, size_t ws_bytes, int n_chunks, void* stream);
+
 /* Expanded weights: the six ternary matrices of a layer expanded once to
  * tensor-core operand form (A8: int8 {-1,0,1}; A16: bf16 w * bf16(s)).
  * bitssm_prepare_weights fills `dst` (bitssm_prepared_size bytes, device,

@@ -93,6 +93,8 @@ _SIGS = {
     "bitssm_forward_state": (_i, [_P_LAYER, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "bitssm_step": (_i, [_P_LAYER, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "bitssm_stack_forward": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "bitssm_forward_host": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _i,
+                                 _vp]),
     "bitssm_forward_launches": (_i, [_P_LAYER, _i]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
                                   ctypes.POINTER(_vp), _i, _vp]),
@@ -245,6 +247,19 @@ def bitssm_stack_forward(layers, x, out, B, L, dtype, act_mode, ws, ws_bytes, st
     _check(_lib.bitssm_stack_forward(arr, len(layers), _ptr(x), _ptr(out), B, L, dtype,
                                      act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitssm_stack_forward")
+
+
+def bitssm_forward_host(layers, x_host, out_host, B, L, dtype, act_mode, x_dev, out_dev, ws,
+                        ws_bytes, n_chunks, stream=None):
+    """x_host / out_host: host tensors (page-locked for overlap); one layer
+    struct or a list of them (a residual stack)."""
+    if isinstance(layers, bitssm_layer):
+        layers = [layers]
+    arr = (bitssm_layer * len(layers))(*layers)
+    _check(_lib.bitssm_forward_host(arr, len(layers), _ptr(x_host), _ptr(out_host), B, L, dtype,
+                                    act_mode, _ptr(x_dev), _ptr(out_dev), _ptr(ws), ws_bytes,
+                                    n_chunks, _stream(stream)),
+           "bitssm_forward_host")
 
 
 def bitssm_prepared_size(layer: bitssm_layer, act_mode) -> int:

@@ -50,7 +50,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "bitssm.cu"), os.path.join(CSRC, "noalloc.cu"), "-o", tmp]
+           os.path.join(CSRC, "bitssm.cu"), os.path.join(CSRC, "noalloc.cu"),
+           os.path.join(CSRC, "host_pipeline.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
