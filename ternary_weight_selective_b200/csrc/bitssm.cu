@@ -129,13 +129,14 @@ int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, c
 
 // W1.58A16 GEMM with exact fp32 group scales (transposed scales in P.s_t).
 // Epilogue warps of the group-scaled GEMM: 8 (two column slices), or 16
-// (four slices of at least 32 columns) for a single 128-wide K group, where
-// the epilogue is the whole cost and the accumulators are few, when the two
-// pipeline stages can hold sixteen output transpose buffers.  The u^2
-// partial sums of ROWSS are laid out for 8.
+// (four slices of at least 32 columns) for a single 128-wide K group (STORE /
+// DELTA with two stages), where the epilogue is the whole cost, when the
+// stages can hold sixteen output transpose buffers (16 warps measured slower
+// for the 32-group x_proj: fewer registers per thread).  The u^2 partial
+// sums of ROWSS are laid out for 8.
 constexpr int gs_nepi(int epi, int bn, int stages) {
-  return ((epi == EPI_STORE || epi == EPI_DELTA) && stages == 2 && bn >= 128 &&
-          16 * kStageFloats * 4 <= stages * (128 * 128 + bn * 128))
+  return (epi == EPI_STORE || epi == EPI_DELTA) && stages == 2 && bn >= 128 &&
+                 16 * kStageFloats * 4 <= stages * (128 * 128 + bn * 128)
              ? 16
              : 8;
 }
@@ -183,7 +184,6 @@ int launch_gemm_gs(const void* A, long lda, const void* W, long ldw, long w_rows
   const bool whole = EPI == EPI_XPROJ_A16;
   if (whole && P.N > 256) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   const int bn = gs_bn(P.N, whole);
-  if (whole && P.R > bn / 2) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (bn == 64) return launch_gemm_gs_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
   if (bn == 128) return launch_gemm_gs_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
   return launch_gemm_gs_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);

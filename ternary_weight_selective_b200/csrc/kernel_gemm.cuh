@@ -578,7 +578,6 @@ __global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
     ternary_gemm_gs_kernel(const __grid_constant__ CUtensorMap mapA,
                            const __grid_constant__ CUtensorMap mapW, GemmParams P) {
   using Cfg = GsConfig<BN, STAGES, NEPI>;
-  static_assert(EPI != EPI_XPROJ_A16 || NEPI == 8, "the x_proj epilogue keeps dt in slice 0");
   constexpr int kPanel = 64;             // bf16 elements per 128-byte panel
   constexpr int kPanelsPerGroup = 2;     // 128-element weight groups
   extern __shared__ uint8_t smem_raw[];
@@ -749,6 +748,7 @@ __global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
         if (EPI == EPI_ROWSS && live) P.ss_part[(long)m * (Cfg::kSlices * gridDim.y) + Cfg::kSlices * blockIdx.y + half] = ss;
       }
     }
+    float ss_dt = 0.f;  // EPI_XPROJ_A16: this slice's sum of dt^2
     if (ok && live) {
       const float rs = P.row_scale != nullptr ? P.row_scale[m] : 1.0f;
       (void)rs;
@@ -769,12 +769,12 @@ __global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
           }
         }
       } else if constexpr (EPI == EPI_XPROJ_A16) {
-        // columns [0,R) dt (all in half 0: R <= BN/2) | [R,R+Ns) B | [R+Ns,R+2Ns) C
+        // columns [0,R) dt | [R,R+Ns) B | [R+Ns,R+2Ns) C; each column slice
+        // sums the squares of the dt values it holds
         const int R = P.R, Ns = P.Ns;
         float t = 0.f;
         for (int j = 0; j < P.ss_nparts; ++j) t += P.ss_in[(long)m * P.ss_nparts + j];
         const float r_u = 1.0f / sqrtf(t / (float)P.ss_count + kEpsNorm);
-        float ss = 0.f;
 #pragma unroll
         for (int j = 0; j < Cfg::kHalf; ++j) {
           const int col = c_base + j;
@@ -783,14 +783,25 @@ __global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
             const __nv_bfloat16 b = __float2bfloat16_rn(v);
             reinterpret_cast<__nv_bfloat16*>(P.out)[(long)m * P.ld_out + col] = b;
             const float vb = __bfloat162float(b);
-            ss = fmaf(vb, vb, ss);
+            ss_dt = fmaf(vb, vb, ss_dt);
           } else if (col < R + Ns) {
             P.Bm[(long)m * Ns + (col - R)] = v;
           } else if (col < R + 2 * Ns) {
             P.Cm[(long)m * Ns + (col - R - Ns)] = v;
           }
         }
-        if (half == 0) P.r_out[m] = 1.0f / sqrtf(ss / (float)R + kEpsNorm);
+      }
+    }
+    if constexpr (EPI == EPI_XPROJ_A16) {
+      // r_dt from the slices' partial sums (the pipeline stages are idle now)
+      float* red = reinterpret_cast<float*>(smem);
+      red[half * 128 + row] = ss_dt;
+      named_bar_sync(1, 32 * NEPI);
+      if (half == 0 && ok && live) {
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < Cfg::kSlices; ++k) s += red[k * 128 + row];
+        P.r_out[m] = 1.0f / sqrtf(s / (float)P.R + kEpsNorm);
       }
     }
   }
