@@ -81,7 +81,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 }
 
 // 2-D tiled load of one box into shared memory; completion is signalled as
-// transaction bytes on `bar`.  No multicast.
+// transaction bytes on `bar`; the data lands in this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             uint32_t bar) {
   asm volatile(
@@ -93,7 +93,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 
 // 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
 // from global into shared memory; completion is signalled as transaction
-// bytes on `bar`.  No multicast.
+// bytes on `bar`; the data lands in this CTA's shared memory only.
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
                                              uint32_t bar) {
   asm volatile(
