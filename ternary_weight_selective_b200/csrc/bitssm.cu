@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -41,15 +42,32 @@ int launch_status() {
   return BITSSM_ERR_CUDA;
 }
 
-int g_num_sms = 0;
+// Opt `kern` into `bytes` of dynamic shared memory on the current device.  The
+// attribute is per device, so it is set once per kernel and device (bit d of
+// `done` marks device d; concurrent first calls may both set it, harmlessly).
+template <typename Kern>
+int set_smem_attr_once(Kern kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return launch_status();
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return BITSSM_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return launch_status();
+  done.fetch_or(bit, std::memory_order_release);
+  return BITSSM_OK;
+}
+
+// SM count of the current device (looked up once per device).
+std::atomic<int> g_num_sms[64];
 int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = g_num_sms[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[dev].store(n, std::memory_order_relaxed);
   }
-  return g_num_sms;
+  return n;
 }
 
 // ------------------------------------------------------------ tensor maps
@@ -96,13 +114,8 @@ int launch_gemm_bn(const void* A, long lda, const void* W, long ldw, long w_rows
   constexpr int kSplit = EPI == EPI_XPROJ_A8 ? 1 : (BN >= 256 ? BN / 128 : 1);
   using Cfg = GemmConfig<BN, kStages, kSplit>;
   auto kern = ternary_gemm_kernel<BN, kStages, EPI, kSplit>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
-        cudaSuccess)
-      return launch_status();
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int rc = set_smem_attr_once(kern, Cfg::kSmemBytes, attr_done)) return rc;
   CUtensorMap mA, mW;
   if (!make_map(&mA, A, false, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (!make_map(&mW, W, false, P.K, w_rows, ldw, BN > 256 ? 256 : BN))
@@ -147,13 +160,8 @@ int launch_gemm_gs_st(const void* A, long lda, const void* W, long ldw, long w_r
   constexpr int kNepi = gs_nepi(EPI, BN, kStages);
   using Cfg = GsConfig<BN, kStages, kNepi>;
   auto kern = ternary_gemm_gs_kernel<BN, kStages, EPI, kNepi>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
-        cudaSuccess)
-      return launch_status();
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int rc = set_smem_attr_once(kern, Cfg::kSmemBytes, attr_done)) return rc;
   CUtensorMap mA, mW;
   if (!make_map(&mA, A, true, P.K, P.M, lda, 128)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (!make_map(&mW, W, true, P.K, w_rows, ldw, BN)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
@@ -273,12 +281,9 @@ int launch_scan_t(const ScanParams& P, cudaStream_t st) {
   constexpr int CE = 128 / TPC;
   constexpr int smem = 2 * ScanStage<CE, FUSED, Tu, Td>::kBytes;
   auto kern = selective_scan_kernel<NPT, FUSED, RV, Tu, Td, Ty, DFIN>;
-  static bool attr_set = false;
-  if (!attr_set && smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return launch_status();
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (smem > 48 * 1024)
+    if (int rc = set_smem_attr_once(kern, smem, attr_done)) return rc;
   dim3 grid((unsigned)((P.E + CE - 1) / CE), (unsigned)P.B);
   kern<<<grid, 128, smem, st>>>(P);
   return launch_status();
@@ -550,12 +555,8 @@ int launch_pre_t(const PreParams& Q, const void* w_in, long ld_in, const void* w
                  int xrows, cudaStream_t st) {
   using Cfg = PreCfg<BN1, K1P, 64>;
   auto kern = bitssm_pre_kernel<Tx, BN1, K1P, 64>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
-      return launch_status();
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int rc = set_smem_attr_once(kern, Cfg::kSmemBytes, attr_done)) return rc;
   CUtensorMap mWin, mWx;
   if (!make_map(&mWin, w_in, false, Q.d, Q.E, ld_in, BN1 > 256 ? 256 : BN1)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (!make_map(&mWx, w_x, false, Q.E, xrows, ld_x, 64)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
@@ -578,12 +579,8 @@ template <int OUT_BF16, int BN, int KP>
 int launch_post_t(const PostParams& Q, const void* w, long ldw, cudaStream_t st) {
   using Cfg = PostCfg<BN, KP>;
   auto kern = bitssm_post_kernel<OUT_BF16, BN, KP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess)
-      return launch_status();
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int rc = set_smem_attr_once(kern, Cfg::kSmemBytes, attr_done)) return rc;
   CUtensorMap mW;
   if (!make_map(&mW, w, false, Q.E, Q.d, ldw, BN)) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   kern<<<(Q.M + 127) / 128, kFusedThreads, Cfg::kSmemBytes, st>>>(mW, Q);

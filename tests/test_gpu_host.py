@@ -59,6 +59,26 @@ def test_host_forward_equals_device_forward(env, wl, n_layers, n_chunks, pinned)
     assert torch.equal(out_dev, ref)
 
 
+def test_host_forward_unprepared_weights(env):
+    """Without prepared weights every chunk expands them into its workspace."""
+    torch, abi, dev = env
+    wl = CASES[0][0]
+    x, layers = S.make_inputs(wl, seed=9)
+    d_l = dev.DeviceLayer(layers[0], abi.A8)
+    B, L, d = x.shape
+    xd = dev.to_device_input(x, abi.BF16)
+    n = abi.bitssm_workspace_size(d_l.layer, B, L, abi.BF16, abi.A8)
+    ws = dev.Workspace(n)
+    ref = torch.zeros_like(xd)
+    abi.bitssm_forward(d_l.layer, xd, ref, None, B, L, abi.BF16, abi.A8, ws.addr, n)
+    xh = xd.cpu().pin_memory()
+    oh = torch.zeros_like(xh).pin_memory()
+    abi.bitssm_forward_host(d_l.layer, xh, oh, B, L, abi.BF16, abi.A8, torch.empty_like(xd),
+                            torch.empty_like(xd), ws.addr, n, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref.cpu())
+
+
 def test_host_forward_argument_errors(env):
     torch, abi, dev = env
     wl = CASES[0][0]
