@@ -247,6 +247,16 @@ int launch_quant_rows(const void* x, int dtype, int M, int K, long ldx, int8_t* 
 
 int launch_row_rms(const void* x, int dtype, int M, int K, long ldx, float* r, cudaStream_t st) {
   if (M == 0) return BITSSM_OK;
+  const int es = dtype == BITSSM_F32 ? 4 : 2;
+  if ((K * es) % 16 == 0 && (ldx * es) % 16 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+    if (dtype == BITSSM_F32)
+      row_rms_vec_kernel<float><<<rows_grid(M), 256, 0, st>>>(reinterpret_cast<const float*>(x), M,
+                                                              K, ldx, r);
+    else
+      row_rms_vec_kernel<__nv_bfloat16><<<rows_grid(M), 256, 0, st>>>(
+          reinterpret_cast<const __nv_bfloat16*>(x), M, K, ldx, r);
+    return launch_status();
+  }
   if (dtype == BITSSM_F32)
     row_rms_kernel<float><<<rows_grid(M), 256, 0, st>>>(reinterpret_cast<const float*>(x), M, K,
                                                         ldx, r);

@@ -224,6 +224,57 @@ __global__ void __launch_bounds__(256) row_rms_kernel(const T* __restrict__ x, i
   }
 }
 
+// Sum of squares of the floats held in one 16-byte vector of T.
+template <typename T>
+__device__ __forceinline__ float vec_sumsq(const uint4 q, float acc);
+template <>
+__device__ __forceinline__ float vec_sumsq<float>(const uint4 q, float acc) {
+  acc = fmaf(__uint_as_float(q.x), __uint_as_float(q.x), acc);
+  acc = fmaf(__uint_as_float(q.y), __uint_as_float(q.y), acc);
+  acc = fmaf(__uint_as_float(q.z), __uint_as_float(q.z), acc);
+  return fmaf(__uint_as_float(q.w), __uint_as_float(q.w), acc);
+}
+template <>
+__device__ __forceinline__ float vec_sumsq<__nv_bfloat16>(const uint4 q, float acc) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xffff0000u);
+    acc = fmaf(a, a, acc);
+    acc = fmaf(b, b, acc);
+  }
+  return acc;
+}
+
+// row_rms_kernel with 16-byte loads: a warp per row, four vectors in flight
+// per lane into four partial sums (rows of K * sizeof(T) bytes, a multiple
+// of 16, at 16-byte aligned starts).
+template <typename T>
+__global__ void __launch_bounds__(256) row_rms_vec_kernel(const T* __restrict__ x, int M, int K,
+                                                          long ldx, float* __restrict__ r) {
+  constexpr int kEpv = 16 / (int)sizeof(T);
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nvec = K / kEpv;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int v = lane;
+    for (; v + 96 < nvec; v += 128) {
+      const uint4 q0 = __ldg(xr + v), q1 = __ldg(xr + v + 32), q2 = __ldg(xr + v + 64),
+                  q3 = __ldg(xr + v + 96);
+      s0 = vec_sumsq<T>(q0, s0);
+      s1 = vec_sumsq<T>(q1, s1);
+      s2 = vec_sumsq<T>(q2, s2);
+      s3 = vec_sumsq<T>(q3, s3);
+    }
+    for (; v < nvec; v += 32) s0 = vec_sumsq<T>(__ldg(xr + v), s0);
+    const float ss = warp_sum((s0 + s1) + (s2 + s3));
+    if (lane == 0) r[row] = 1.0f / sqrtf(ss / (float)K + kEpsNorm);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Absmean ternary packing (BitNet b1.58 weights; grouped scales: Ternary
 // Mamba abstract).  s = mean|W| summed in float64 and rounded to float;
