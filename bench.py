@@ -132,13 +132,16 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- byte counts
 
-def scan_bytes_per_token(E, N, R_pad, a16=False):
+def scan_bytes_per_token(E, N, R_pad, a16=False, predelta=False):
     """Algorithmic HBM bytes of the scan kernel per token.
     A8 (Delta-up fused): read u (int16 accumulators + one fp32 scale), the
     Delta-down codes and their factor, B and C (fp32); write y (fp32).
+    A8 with delta formed before the scan: delta (fp32) instead of the codes.
     A16: read u (bf16), delta (fp32), B and C; write y (bf16)."""
     if a16:
         return E * 2 + E * 4 + 2 * N * 4 + E * 2
+    if predelta:
+        return E * 2 + 4 + E * 4 + 2 * N * 4 + E * 4
     return E * 2 + 4 + R_pad + 4 + 2 * N * 4 + E * 4
 
 
@@ -226,7 +229,7 @@ def run_ours(args):
                 d_l.unprepare()
         nbytes = abi.bitssm_workspace_size(dl[0].layer, B, L, dtype, act)
         ws = dev.Workspace(nbytes)
-        nl = abi.bitssm_forward_launches(dl[0].layer, act)
+        nl = abi.bitssm_forward_launches(dl[0].layer, B, L, act)
         per_step = n_layers * (nl + 1)
 
         def forward(evs=None):
@@ -420,6 +423,9 @@ def run_ours(args):
     if act == abi.A8 and nl == 3:
         names = ["expand_weights", "bitssm_pre(quant_x+in_proj+x_proj)",
                  "selective_scan_fused_dt", "bitssm_post(quant_y+out_proj)"]
+    elif act == abi.A8 and nl == 4:
+        names = ["expand_weights", "bitssm_pre(quant_x+in_proj+x_proj)",
+                 "gemm_dt_proj(+softplus)", "selective_scan", "bitssm_post(quant_y+out_proj)"]
     elif act == abi.A8:
         names = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_x_proj",
                  "selective_scan_fused_dt", "quant_rows_y", "gemm_out_proj"]
@@ -442,7 +448,8 @@ def run_ours(args):
         t_s = avg_kernel_ms[dom] / 1e3
         achieved = exps / t_s / 1e12
         peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e12
-        hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp, act == abi.A16)
+        hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp, act == abi.A16,
+                                             act == abi.A8 and nl == 4)
         roof = {"kernel": names[dom], "bound": "alu", "unit": "Tex2/s",
                 "achieved": round(achieved, 4), "peak": round(peak, 4),
                 "frac": round(achieved / peak, 4),

@@ -230,14 +230,17 @@ int bitssm_workspace_size(const bitssm_layer* p, int B, int L, int dtype, int ac
 int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* residual, int B,
                    int L, int dtype, int act_mode, void* ws, size_t ws_bytes, void* stream);
 
-/* Number of kernels one bitssm_forward call launches for this layer and act
- * mode, or -1 for a bad argument.  A8 with d_model in {128, 256}, d_inner in
- * {256, 512} and dt_rank + 2 d_state <= 64: 3 (pre = quantise x + in_proj +
- * x_proj; scan with Delta-up fused; post = quantise y + out_proj); other A8
- * shapes: 6 (quantise x, in_proj, x_proj, scan, quantise y, out_proj).
- * A16: 7 (RMS of x, in_proj, x_proj, dt_proj, scan, RMS of y, out_proj).
- * Plus 1 (first) for the weight expansion when `prepared` is NULL. */
-int bitssm_forward_launches(const bitssm_layer* p, int act_mode);
+/* Number of kernels one bitssm_forward call over B sequences of length L
+ * launches for this layer and act mode, or -1 for a bad argument.  A8 with
+ * d_model in {128, 256}, d_inner in {256, 512} and dt_rank + 2 d_state <= 64:
+ * 3 (pre = quantise x + in_proj + x_proj; scan with Delta-up fused; post =
+ * quantise y + out_proj), or 4 when B * d_inner is small (below 24 x the SM
+ * count): pre, Delta-up + softplus as an int8 GEMM writing delta, the scan
+ * reading it, post.  Other A8 shapes: 6 (quantise x, in_proj, x_proj, scan,
+ * quantise y, out_proj).  A16: 7 (RMS of x, in_proj, x_proj, dt_proj, scan,
+ * RMS of y, out_proj).  Plus 1 (first) for the weight expansion when
+ * `prepared` is NULL. */
+int bitssm_forward_launches(const bitssm_layer* p, int B, int L, int act_mode);
 
 /* bitssm_forward, additionally recording events[i] (cudaEvent_t handles
  * created by the caller, passed as void*) on `stream` before the i-th kernel
@@ -323,7 +326,9 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
  *        u = u_i16 * u_scale[t], u_scale float [T]),
  *        q_u int8 [T, ld_qu], deq_u float [T], Bm float [T, N],
  *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],
- *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]
+ *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]; delta float
+ *        [T, E] only when the forward forms it by a GEMM before the scan
+ *        (see bitssm_forward_launches)
  *   A16: r_x float [T], u bf16 [T, E], dt_low bf16 [T, R], r_dt float [T],
  *        Bm, Cm float [T, N], delta float [T, E] (= softplus(delta_raw +
  *        dt_bias), formed in the dt_proj epilogue), y bf16 [T, E],

@@ -95,7 +95,7 @@ _SIGS = {
     "bitssm_stack_forward": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _sz, _vp]),
     "bitssm_forward_host": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _i,
                                  _vp]),
-    "bitssm_forward_launches": (_i, [_P_LAYER, _i]),
+    "bitssm_forward_launches": (_i, [_P_LAYER, _i, _i, _i]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
                                   ctypes.POINTER(_vp), _i, _vp]),
     "bitssm_prepared_size": (_i, [_P_LAYER, _i, ctypes.POINTER(_sz)]),
@@ -226,8 +226,8 @@ def bitssm_step(layer: bitssm_layer, x, out, residual, h, B, dtype, act_mode, ws
            "bitssm_step")
 
 
-def bitssm_forward_launches(layer: bitssm_layer, act_mode) -> int:
-    n = _lib.bitssm_forward_launches(ctypes.byref(layer), act_mode)
+def bitssm_forward_launches(layer: bitssm_layer, B, L, act_mode) -> int:
+    n = _lib.bitssm_forward_launches(ctypes.byref(layer), B, L, act_mode)
     if n < 0:
         raise BitssmError(ERR_INVALID_ARG, "bitssm_forward_launches")
     return n

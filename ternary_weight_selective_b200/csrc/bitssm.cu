@@ -105,13 +105,21 @@ bool make_map(CUtensorMap* map, const void* ptr, bool bf16, long k, long rows, l
 }
 
 // ------------------------------------------------------------ GEMM launch
-template <int BN, int EPI>
+// kStagesWant = 0: as many pipeline stages (up to 4) as 200 KB holds.  The
+// delta GEMM (K <= 128: one panel) takes two (room for the output transpose
+// buffers of its 16 epilogue warps), so two CTAs share an SM and one's
+// epilogue stores overlap another's loads.
+template <int BN, int EPI, int kStagesWant = 0>
 int launch_gemm_bn(const void* A, long lda, const void* W, long ldw, long w_rows,
                    const GemmParams& P, cudaStream_t st) {
   constexpr int kStage = 128 * 128 + BN * 128;
-  constexpr int kStages = (200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage);
-  // epilogue warps per TMEM quadrant: 128-column slices (x_proj keeps whole rows)
-  constexpr int kSplit = EPI == EPI_XPROJ_A8 ? 1 : (BN >= 256 ? BN / 128 : 1);
+  constexpr int kStages =
+      kStagesWant > 0 ? kStagesWant : ((200 * 1024 / kStage) >= 4 ? 4 : (200 * 1024 / kStage));
+  // epilogue warps per TMEM quadrant: 128-column slices (x_proj keeps whole
+  // rows); the delta GEMM, bound by its softplus epilogue, 64-column slices
+  constexpr int kSplit = EPI == EPI_XPROJ_A8 ? 1
+                         : EPI == EPI_DELTA  ? BN / 64
+                                             : (BN >= 256 ? BN / 128 : 1);
   using Cfg = GemmConfig<BN, kStages, kSplit>;
   auto kern = ternary_gemm_kernel<BN, kStages, EPI, kSplit>;
   static std::atomic<uint64_t> attr_done{0};
@@ -130,6 +138,11 @@ int launch_gemm_bn(const void* A, long lda, const void* W, long ldw, long w_rows
 template <int EPI>
 int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, const GemmParams& P,
                 cudaStream_t st) {
+  if constexpr (EPI == EPI_DELTA) {
+    if (P.K > 128) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+    if (P.N <= 128) return launch_gemm_bn<128, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+    return launch_gemm_bn<256, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+  }
   const int need = EPI == EPI_STORE ? (P.N < 256 ? P.N : 256) : P.N;
   if (need <= 64) return launch_gemm_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
   if (need <= 128) return launch_gemm_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
@@ -373,6 +386,7 @@ struct LayerPlan {
   bitssm_ws_view v;
   size_t ss_u;             // A16 partial sums
   int ss_parts;
+  bool predelta;           // A8 fused: delta formed by a GEMM before the scan
   size_t total;
 };
 
@@ -408,6 +422,20 @@ int layer_supported(const bitssm_layer* p, int act_mode) {
     if (p->dt_rank + 2 * p->d_state > 256) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   }
   return BITSSM_OK;
+}
+
+// The A8 layer runs as the fused three-kernel path for these shapes.
+bool a8_fused(const LayerPlan& P) {
+  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64 && P.R <= 64;
+}
+
+// Fused A8 with few channels (B * E below ~96 per SM sub-partition, where the
+// fused scan would take 4 states per thread): the Delta-up projection and the
+// softplus run first as an int8 GEMM writing delta, and the scan reads it
+// ready-made (the scan then spends its issue slots on the recurrence alone).
+bool a8_predelta(const LayerPlan& P, int B) {
+  const long want = (long)num_sms() * 4 * 48;
+  return !P.a16 && a8_fused(P) && 2L * B * P.E < want;
 }
 
 LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool prepared) {
@@ -480,6 +508,8 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
     v.y = take(T * P.E * 2);
     v.r_y = take(T * 4);
   }
+  P.predelta = a8_predelta(P, B);
+  if (P.predelta) v.delta = take(T * P.E * 4);
   P.total = a;
   return P;
 }
@@ -556,9 +586,6 @@ T* at(void* base, size_t off) {
 
 // Whether the A8 layer runs as the fused pre kernel + scan + post kernel:
 // d_model of 128 or 256, d_inner of 256 or 512, dt_rank + 2 d_state <= 64.
-bool a8_fused(const LayerPlan& P) {
-  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64 && P.R <= 64;
-}
 
 template <typename Tx, int BN1, int K1P>
 int launch_pre_t(const PreParams& Q, const void* w_in, long ld_in, const void* w_x, long ld_x,
@@ -633,6 +660,19 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
              : launch_pre<__nv_bfloat16>(Q, wexp + P.w_in, P.ld_d, wexp + P.w_x, P.ld_E, P.xrows, st);
     if (rc) return rc;
   }
+  if (P.predelta) {  // delta = softplus(s_up * deq_dt * (W_up . q_dt) + bias), int8 GEMM
+    mk.mark();
+    GemmParams G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = P.T; G.N = P.E; G.K = P.ld_R;
+    G.out_dtype = BITSSM_F32;
+    G.alpha = p->dt_up.scales;
+    G.row_scale = at<float>(ws, v.deq_dt);
+    G.bias = p->dt_bias;
+    G.out = at<float>(ws, v.delta); G.ld_out = P.E;
+    rc = launch_gemm<EPI_DELTA>(at<int8_t>(ws, v.q_dt), P.ld_R, wexp + P.w_up, P.ld_R, P.E, G, st);
+    if (rc) return rc;
+  }
   mk.mark();
   {
     ScanParams S;
@@ -648,7 +688,12 @@ int forward_a8_fused(const bitssm_layer* p, const LayerPlan& P, const uint8_t* w
     S.y = at<float>(ws, v.y);
     S.B = B; S.L = L; S.E = P.E;
     S.h0 = h; S.h_last = h;  // carried state (nullable): read, then overwritten
-    rc = launch_scan<true, int16_t, float, float>(S, st);
+    if (P.predelta) {
+      S.delta_raw = at<float>(ws, v.delta);  // already delta
+      rc = launch_scan<false, int16_t, float, float, true>(S, st);
+    } else {
+      rc = launch_scan<true, int16_t, float, float>(S, st);
+    }
     if (rc) return rc;
   }
   mk.mark();
@@ -1139,18 +1184,19 @@ int bitssm_step(const bitssm_layer* p, const void* x, void* out, const void* res
   return bitssm_forward_state(p, x, out, residual, h, B, 1, dtype, act_mode, ws, ws_bytes, stream);
 }
 
-int bitssm_forward_launches(const bitssm_layer* p, int act_mode) {
-  if (p == nullptr || (act_mode != BITSSM_A8 && act_mode != BITSSM_A16)) return -1;
+int bitssm_forward_launches(const bitssm_layer* p, int B, int L, int act_mode) {
+  if (p == nullptr || B < 0 || L < 0 || (act_mode != BITSSM_A8 && act_mode != BITSSM_A16))
+    return -1;
   const int expand = p->prepared != nullptr ? 0 : 1;
   if (act_mode == BITSSM_A16) return expand + 7;
-  const LayerPlan P = plan_layer(p, 1, 1, act_mode, p->prepared != nullptr);
-  return expand + (a8_fused(P) ? 3 : 6);
+  const LayerPlan P = plan_layer(p, B, L, act_mode, p->prepared != nullptr);
+  return expand + (a8_fused(P) ? (P.predelta ? 4 : 3) : 6);
 }
 
 int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const void* residual,
                          int B, int L, int dtype, int act_mode, void* ws, size_t ws_bytes,
                          void* const* events, int n_events, void* stream) {
-  const int nl = bitssm_forward_launches(p, act_mode);
+  const int nl = bitssm_forward_launches(p, B, L, act_mode);
   if (nl < 0 || events == nullptr || n_events < nl + 1) return BITSSM_ERR_INVALID_ARG;
   for (int i = 0; i <= nl; ++i)
     if (events[i] == nullptr) return BITSSM_ERR_INVALID_ARG;

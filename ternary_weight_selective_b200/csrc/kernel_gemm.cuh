@@ -32,7 +32,8 @@ enum EpiKind : int {
   EPI_XPROJ_A8 = 2,   // A8 x_proj: dt codes + deq_dt from the int32 row, B and C (f32)
   EPI_ROWSS = 3,      // A16 in_proj: u (bf16) = acc * r_x + partial sum(u^2) per tile
   EPI_XPROJ_A16 = 4,  // A16 x_proj: dt_low (bf16) + r_dt, B and C (f32)
-  EPI_DELTA = 5,      // A16 dt_proj: delta = softplus(acc * row_scale[m] + bias[n]) -> f32
+  EPI_DELTA = 5,      // dt_proj: delta = softplus(acc * alpha * row_scale[m] + bias[n]) -> f32
+                      // (A16: the group-scaled kernel, alpha = 1; A8: the int8 kernel)
 };
 
 struct GemmParams {
@@ -370,6 +371,25 @@ __global__ void __launch_bounds__(GemmConfig<BN, STAGES, CSPLIT>::kThreads, 1)
           if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
           store16(P.out, idx, P.out_dtype, v, valid);
         }
+      }
+    } else if constexpr (EPI == EPI_DELTA) {
+      // delta = softplus(acc * alpha * row_scale + bias) in fp32, stored
+      // through the per-warp transpose buffers in the idle pipeline stages
+      // (every lane takes part; rows >= M are skipped inside the store)
+      static_assert(4 * CSPLIT * kStageFloats * 4 <= STAGES * Cfg::kStageBytes, "output staging");
+      const float f = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;
+      float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * kStageFloats;
+#pragma unroll 1
+      for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(trow + c0, r);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = n0 + cs + c0 + j;
+          v[j] = softplus_fast(fmaf(i2f_exact((int)r[j]), f, col < P.N ? __ldg(P.bias + col) : 0.f));
+        }
+        if (ok) warp_store_block<0>(stg, v, lane, P.out, nullptr, P.ld_out, m0 + q * 32, n0 + cs + c0, P.M, P.N);
       }
     } else if constexpr (EPI == EPI_QUANT_ROW) {
       // whole row in this tile (n0 == 0, N <= BN).  Pass 1: max|acc| in

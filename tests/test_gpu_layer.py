@@ -85,6 +85,10 @@ def a8_stage_checks(env, x, lw, ws, dl, out_gpu, dtype):
     # scan, teacher-forced on the GPU's own stage outputs
     delta_raw = O.int_gemm(q_dt[:, :R], P.Wq["W_dt_up"]) * np.float64(P.s["W_dt_up"]) * deq_dt[:, None]
     delta = O.softplus(delta_raw + P.dt_bias[None])
+    if v.delta != 2**64 - 1:
+        # delta formed by the int8 GEMM before the scan (small B * E): the
+        # exact accumulator times the float32 factor, then the softplus
+        assert rel_err(g(v.delta, torch.float32, (T, E)), delta) <= TOL_F32
     y_tf, _ = O.selective_scan(u.reshape(B, L, E), delta.reshape(B, L, E), P.A,
                                Bm.reshape(B, L, N), Cm.reshape(B, L, N), P.D)
     y = g(v.y, torch.float32, (T, E))
@@ -149,7 +153,10 @@ def test_ragged_shapes_a8_fused(env, B, L, dt):
     if dt == "f32":
         x = S.random_rows(B + L, B * L, 256).reshape(B, L, 256)
     out, ws, dl = run_layers(env, x, layers, abi.A8, dtype)
-    assert abi.bitssm_forward_launches(dl[0].layer, abi.A8) == 4
+    # prepared weights off: expansion + pre + scan + post, plus the delta GEMM
+    # when B * E is small (the fused scan would run 4 states per thread)
+    predelta = 2 * B * 512 < 148 * 4 * 48
+    assert abi.bitssm_forward_launches(dl[0].layer, B, L, abi.A8) == (5 if predelta else 4)
     a8_stage_checks(env, x, layers[0], ws, dl[0], out, dtype)
 
 
