@@ -196,6 +196,9 @@ int launch_gemm_gs_bn(const void* A, long lda, const void* W, long ldw, long w_r
 // one tile (and the dt columns within the first half).
 inline int gs_bn(int N, bool whole_row) {
   const int need = whole_row ? N : (N < 256 ? N : 256);
+  // a whole-row tile of up to 160 columns (x_proj at dt_rank 128, d_state 16)
+  // keeps the MMA and the per-group promotion to the columns that exist
+  if (whole_row && need > 128 && need <= 160) return 160;
   return need <= 64 ? 64 : need <= 128 ? 128 : 256;
 }
 
@@ -207,6 +210,9 @@ int launch_gemm_gs(const void* A, long lda, const void* W, long ldw, long w_rows
   const int bn = gs_bn(P.N, whole);
   if (bn == 64) return launch_gemm_gs_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
   if (bn == 128) return launch_gemm_gs_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
+  if constexpr (EPI == EPI_XPROJ_A16) {
+    if (bn == 160) return launch_gemm_gs_bn<160, EPI>(A, lda, W, ldw, w_rows, P, st);
+  }
   return launch_gemm_gs_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);
 }
 

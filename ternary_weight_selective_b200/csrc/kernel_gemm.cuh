@@ -589,7 +589,9 @@ struct GsConfig {
   static constexpr int kHalf = BN / kSlices;  // columns per epilogue warp
   static constexpr int kThreads = 64 + 32 * NEPI;
   static_assert(NEPI == 8 || NEPI == 16, "NEPI");
-  static_assert(BN % (32 * kSlices) == 0 && BN >= 32 && BN <= 256, "BN");
+  // slices of whole 16-column TMEM loads (the transposed-store epilogues also
+  // need whole 32-column blocks, checked where they are used)
+  static_assert(BN % (16 * kSlices) == 0 && BN >= 32 && BN <= 256, "BN");
   static_assert(NEPI * kStageFloats * 4 <= STAGES * kStageBytes, "output staging");
 };
 
@@ -738,6 +740,7 @@ __global__ void __launch_bounds__(GsConfig<BN, STAGES, NEPI>::kThreads, 1)
     // per-warp transpose buffer in the (now idle) pipeline stages.  Every
     // lane takes part (rows >= M are skipped inside the store).
     if constexpr (EPI == EPI_STORE || EPI == EPI_ROWSS || EPI == EPI_DELTA) {
+      static_assert(Cfg::kHalf % 32 == 0, "transposed stores take 32-column blocks");
       const int odt = EPI == EPI_ROWSS ? 1 : EPI == EPI_DELTA ? 0 : P.out_dtype;
       if (ok && odt != 2) {
         const float rs = (live && P.row_scale != nullptr) ? P.row_scale[m] : 1.0f;
