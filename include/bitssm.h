@@ -116,10 +116,20 @@ const char* bitssm_last_error(void);
 
 /* Reads the device error word of the current device into *flags (bit 0: a
  * TMA wait ran out, bit 1: an MMA-completion wait ran out, bit 2: an
- * epilogue wait ran out) after synchronising the device; clears it when
- * `clear` is non-zero.  Returns BITSSM_OK, or BITSSM_ERR_TIMEOUT when any
- * bit was set, or BITSSM_ERR_CUDA. */
+ * epilogue wait ran out, bit 3: the wait of bitssm_selftest_wait) after
+ * synchronising the device; clears it when `clear` is non-zero.  Returns
+ * BITSSM_OK, or BITSSM_ERR_TIMEOUT when any bit was set, or BITSSM_ERR_CUDA. */
 int bitssm_device_error(unsigned int* flags, int clear);
+
+/* Diagnostic of the failure-detection path: one kernel waits, through the
+ * same bounded mbarrier wait every kernel of the library uses, on a barrier
+ * that nothing completes, with a limit of limit_us microseconds (1 ..
+ * 1,000,000) instead of the library's 2 s; it gives up, sets bit 3 of the
+ * device error word and returns, leaving the context usable.  Asynchronous on
+ * `stream`.  BITSSM_ERR_INVALID_ARG for a limit out of range.  The pages have
+ * no counterpart; it exists so the error path can be exercised without a
+ * fault. */
+int bitssm_selftest_wait(unsigned int limit_us, void* stream);
 
 /* ---------------------------------------------------------------------
  * Weight packing (offline).  Absmean ternarisation of the BitNet b1.58

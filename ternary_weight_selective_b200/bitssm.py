@@ -96,6 +96,7 @@ _SIGS = {
     "bitssm_forward_host": (_i, [_P_LAYER, _i, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _i,
                                  _vp]),
     "bitssm_forward_launches": (_i, [_P_LAYER, _i, _i, _i]),
+    "bitssm_selftest_wait": (_i, [ctypes.c_uint, _vp]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
                                   ctypes.POINTER(_vp), _i, _vp]),
     "bitssm_prepared_size": (_i, [_P_LAYER, _i, ctypes.POINTER(_sz)]),
@@ -224,6 +225,10 @@ def bitssm_step(layer: bitssm_layer, x, out, residual, h, B, dtype, act_mode, ws
     _check(_lib.bitssm_step(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual), _ptr(h), B,
                             dtype, act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitssm_step")
+
+
+def bitssm_selftest_wait(limit_us: int, stream=None):
+    _check(_lib.bitssm_selftest_wait(limit_us, _stream(stream)), "bitssm_selftest_wait")
 
 
 def bitssm_forward_launches(layer: bitssm_layer, B, L, act_mode) -> int:

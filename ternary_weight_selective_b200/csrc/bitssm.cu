@@ -906,6 +906,21 @@ void set_last_error_message(const char* msg) {
 
 using namespace bitssm;
 
+namespace bitssm {
+// Self-test of the bounded-wait path: one thread waits on an mbarrier that
+// nothing arrives on, with the given limit; the wait gives up and raises
+// DEVFLAG_TIMEOUT_SELFTEST in the device error word, and the kernel returns.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    (void)mbar_wait_for(b, 0u, DEVFLAG_TIMEOUT_SELFTEST, limit_ns);
+  }
+}
+}  // namespace bitssm
+
 extern "C" {
 
 int bitssm_version(void) { return BITSSM_ABI_VERSION; }
@@ -923,6 +938,12 @@ const char* bitssm_status_string(int status) {
     case BITSSM_ERR_DEVICE_FLAG: return "device-side check failed";
     default: return "unknown status";
   }
+}
+
+int bitssm_selftest_wait(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return BITSSM_ERR_INVALID_ARG;
+  bitssm::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us);
+  return launch_status();
 }
 
 int bitssm_device_error(unsigned int* flags, int clear) {

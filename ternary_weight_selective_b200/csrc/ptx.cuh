@@ -18,6 +18,7 @@ enum : unsigned int {
   DEVFLAG_TIMEOUT_TMA = 1u,
   DEVFLAG_TIMEOUT_MMA = 2u,
   DEVFLAG_TIMEOUT_EPI = 4u,
+  DEVFLAG_TIMEOUT_SELFTEST = 8u,  // the wait of bitssm_selftest_wait
 };
 
 // Wait limit of every mbarrier wait: 2 s of %globaltimer.
@@ -61,18 +62,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int flag) {
+// Bounded wait for the phase with the given parity to complete: false, with
+// `flag` raised in the device error word, once `limit_ns` of %globaltimer
+// have passed.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, unsigned int flag,
+                                              unsigned long long limit_ns) {
   for (int i = 0; i < 128; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       raise_flag(flag);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int flag) {
+  return mbar_wait_for(bar, parity, flag, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA
