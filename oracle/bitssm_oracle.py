@@ -32,6 +32,13 @@ Sources (page title, then the part of the page):
 * [SSDi8] "SSDi8: Accurate and Efficient 8-bit Quantization for State Space
   Duality", abstract: reuse of quantised activations across modules.
 
+The Mamba-1 block form (``bitssm_block_a8``: a depthwise causal conv1d and a
+SiLU on the in_proj branch, a SiLU gate from a second in_proj branch z on the
+scan output) is named by none of the pages; it is the block that the pages'
+Mamba checkpoints carry around the same selective scan (the [TernaryMamba]
+abstract quantises Mamba models), with every projection a ternary BitLinear
+as in the mixer.
+
 The pages name these operations but print no formula.  The formulas used here
 are the BitNet b1.58 definitions the pages refer to by name (absmean ternary
 weights, absmax int8 activations with Q = 127, int32 accumulation, rescale by
@@ -305,6 +312,43 @@ def selective_scan_associative(u, delta, A, Bm, Cm, D, h0=None, chunk=16):
 
 
 # ---------------------------------------------------------------------------
+# Mamba-1 block pieces: depthwise causal conv1d and SiLU
+# ---------------------------------------------------------------------------
+
+def causal_conv1d(v: np.ndarray, w: np.ndarray, b=None) -> np.ndarray:
+    """Depthwise causal convolution along time, one filter per channel.
+
+    v [B, L, E], w [E, K], b [E] or None.  out[:, l, e] = b[e] +
+    sum_{k=0}^{K-1} w[e, k] * v[:, l - (K-1) + k, e], terms with a negative
+    time index dropped (zero padding on the left): tap K-1 multiplies the
+    current step, tap 0 the step K-1 earlier.  This is a width-K conv with
+    K-1 zeros of left padding whose output is cut to the first L steps, the
+    usual causal form.  float64.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Bsz, L, E = v.shape
+    K = w.shape[1]
+    out = np.zeros_like(v)
+    if b is not None:
+        out += np.asarray(b, dtype=np.float64)[None, None, :]
+    for k in range(K):
+        shift = K - 1 - k          # how many steps back tap k looks
+        if shift >= L:
+            continue
+        out[:, shift:, :] += w[None, None, :, k] * v[:, :L - shift, :]
+    return out
+
+
+def silu(v: np.ndarray) -> np.ndarray:
+    """SiLU(v) = v * sigmoid(v) = v / (1 + e^-v), float64; for v < 0 written
+    as v e^v / (1 + e^v) so that e^-v cannot overflow."""
+    v = np.asarray(v, dtype=np.float64)
+    e = np.exp(-np.abs(v))                     # in (0, 1]
+    return np.where(v >= 0, v / (1.0 + e), v * e / (1.0 + e))
+
+
+# ---------------------------------------------------------------------------
 # The BitSSM mixer and the stack
 # ---------------------------------------------------------------------------
 
@@ -323,6 +367,13 @@ class TernaryLayer:
         self.dt_bias = np.asarray(lw.dt_bias, dtype=np.float64)
         self.R = lw.W_dt_down.shape[0]
         self.N = lw.W_B.shape[0]
+        # Mamba-1 block extras (None for the mixer)
+        self.block = getattr(lw, "W_z", None) is not None
+        if self.block:
+            self.Wq["W_z"], self.s["W_z"] = absmean_ternary(lw.W_z, group)
+            self.conv_w = np.asarray(lw.conv_w, dtype=np.float64)
+            self.conv_b = (np.zeros(self.conv_w.shape[0]) if lw.conv_b is None
+                           else np.asarray(lw.conv_b, dtype=np.float64))
 
 
 def bitssm_layer_a8(x: np.ndarray, P: TernaryLayer, h0=None) -> tuple[np.ndarray, dict]:
@@ -395,7 +446,61 @@ def bitssm_layer_a16(x: np.ndarray, P: TernaryLayer, h0=None) -> tuple[np.ndarra
     return out.reshape(Bsz, L, -1), stages
 
 
+def bitssm_block_a8(x: np.ndarray, P: TernaryLayer) -> tuple[np.ndarray, dict]:
+    """The mixer in Mamba-1 block form with int8 activations, x [B, L, d] ->
+    out [B, L, d], from a zero state.
+
+    Steps (the mixer of ``bitssm_layer_a8`` with three additions):
+      1. x-branch and gate branch: u_pre = BitLinear(x; W_in), z =
+         BitLinear(x; W_z), two ternary projections of the same int8 codes of
+         x (the two halves of Mamba's in_proj, each with its own absmean
+         scale);
+      2. u = SiLU(causal_conv1d(u_pre; conv_w, conv_b));
+      3. x_proj (Delta-down | B | C) is a BitLinear on u; u is no longer a
+         scaled integer row, so its codes are taken from its float32 value
+         (``bitlinear_a8``), not from an integer row;
+      4. Delta-up, softplus and the selective scan as in the mixer, on u;
+      5. the gate: y_g = y * SiLU(z), and out_proj is a BitLinear on y_g.
+    Readings: the conv acts on the full-precision u_pre; the codes of u and of
+    y_g are decided in float32 (the precision of the kernel path).
+    """
+    if not P.block:
+        raise ValueError("layer has no block weights")
+    Bsz, L, d = x.shape
+    T = Bsz * L
+    xt = np.asarray(x).reshape(T, d)
+    u_pre, st_in = bitlinear_a8(xt, P.Wq["W_in"], P.s["W_in"])
+    acc_z = int_gemm(st_in["q"], P.Wq["W_z"])
+    z = acc_z.astype(np.float64) * np.float64(P.s["W_z"]) * st_in["deq"][:, None]
+    E = u_pre.shape[1]
+    u = silu(causal_conv1d(u_pre.reshape(Bsz, L, E), P.conv_w, P.conv_b)).reshape(T, E)
+    W_x = np.concatenate([P.Wq["W_dt_down"], P.Wq["W_B"], P.Wq["W_C"]], axis=0)
+    _, st_x = bitlinear_a8(u, W_x, 1.0)
+    acc_x, deq_u = st_x["acc"], st_x["deq"]
+    R, N = P.R, P.N
+    Bm = acc_x[:, R:R + N] * np.float64(P.s["W_B"]) * deq_u[:, None]
+    Cm = acc_x[:, R + N:R + 2 * N] * np.float64(P.s["W_C"]) * deq_u[:, None]
+    c_dt = np.float64(P.s["W_dt_down"]) * deq_u
+    delta_raw, st_dt = bitlinear_a8_int_input(acc_x[:, :R], c_dt, P.Wq["W_dt_up"],
+                                              P.s["W_dt_up"])
+    delta = softplus(delta_raw + P.dt_bias[None])
+    y, h_last = selective_scan(u.reshape(Bsz, L, E), delta.reshape(Bsz, L, E), P.A,
+                               Bm.reshape(Bsz, L, N), Cm.reshape(Bsz, L, N), P.D)
+    y = y.reshape(T, E)
+    yg = y * silu(z)
+    out, st_out = bitlinear_a8(yg, P.Wq["W_out"], P.s["W_out"])
+    stages = dict(q_x=st_in["q"], deq_x=st_in["deq"], u_pre=u_pre, z=z, u=u,
+                  q_u=st_x["q"], deq_u=deq_u, acc_x=acc_x, Bm=Bm, Cm=Cm,
+                  q_dt=st_dt["q"], deq_dt=st_dt["deq"], delta=delta, y=y, yg=yg,
+                  q_y=st_out["q"], deq_y=st_out["deq"], h_last=h_last)
+    return out.reshape(Bsz, L, -1), stages
+
+
 def bitssm_layer(x, P: TernaryLayer, h0=None):
+    if getattr(P, "block", False):
+        if P.act_mode != "A8" or h0 is not None:
+            raise NotImplementedError("block form: A8 from a zero state only")
+        return bitssm_block_a8(x, P)
     if P.act_mode == "A16":
         return bitssm_layer_a16(x, P, h0)
     return bitssm_layer_a8(x, P, h0)

@@ -21,13 +21,20 @@ Workloads (the shapes the pages train and evaluate at):
   Space Models" (abstract)
 * ``long16k``  B=16, L=16384, the TriSSM mixer on a long sequence, input =
   embeddings of a uniform id stream
+* ``trissm_block``  the ``trissm`` shapes as a Mamba-1 block: a depthwise
+  causal conv1d of width 4 and a SiLU on the in_proj branch, and a SiLU gate
+  from a second (ternary) in_proj branch z on the scan output
 
 Draw order for seed s (numpy PCG64 ``default_rng(s)``): the input first
 (x ~ N(0,1), or the embedding table ~ N(0,1) followed by the ids), then for
 each layer W_in, W_dt_down, W_B, W_C, W_dt_up, W_out (all N(0, 0.02)),
 A_log ~ U(log 1, log 16), dt_bias ~ U(log 1e-3, log 1e-1); D = 1.
-A = -exp(A_log).  Weights are returned as float32 full-precision matrices;
-ternarisation is the method's business, not this module's.
+A = -exp(A_log).  Block workloads then draw, per layer, W_z ~ N(0, 0.02)
+[d_inner, d_model], the conv taps ~ U(-1/sqrt(w), 1/sqrt(w)) [d_inner, w]
+and the conv bias ~ U(-1/sqrt(w), 1/sqrt(w)) [d_inner] (w = d_conv; the
+usual fan-in bound of a depthwise conv).  Weights are returned as float32
+full-precision matrices; ternarisation is the method's business, not this
+module's.
 """
 
 from __future__ import annotations
@@ -53,6 +60,8 @@ class Workload:
     act_mode: str      # "A8" (int8 activation codes) or "A16" (bf16, grouped scales)
     layers: int = 1
     source: str = "gauss"  # "gauss": x ~ N(0,1); "embed": x = E[ids]
+    block: bool = False    # Mamba-1 block: conv1d + SiLU on u, SiLU(z) gate on y
+    d_conv: int = 4        # conv width (block workloads)
 
     @property
     def tokens(self) -> int:
@@ -71,6 +80,8 @@ WORKLOADS = {
     "long16k": Workload("long16k", 16, 16384, 256, 512, 16, 16, "bf16", "A8", source="embed"),
     # decode: one token for each of 64 sequences, the state carried in h
     "trissm_decode": Workload("trissm_decode", 64, 1, 256, 512, 16, 16, "bf16", "A8"),
+    # the Mamba-1 block form of the trissm mixer (conv1d, SiLU, z gate)
+    "trissm_block": Workload("trissm_block", 64, 256, 256, 512, 16, 16, "bf16", "A8", block=True),
 }
 
 
@@ -109,6 +120,9 @@ class LayerWeights:
     A: np.ndarray          # [d_inner, d_state], negative
     D: np.ndarray          # [d_inner]
     dt_bias: np.ndarray    # [d_inner]
+    W_z: np.ndarray | None = None     # [d_inner, d_model], block only
+    conv_w: np.ndarray | None = None  # [d_inner, d_conv], block only
+    conv_b: np.ndarray | None = None  # [d_inner], block only
 
 
 def _layer(rng: np.random.Generator, wl: Workload) -> LayerWeights:
@@ -127,8 +141,15 @@ def _layer(rng: np.random.Generator, wl: Workload) -> LayerWeights:
     dt_bias = rng.uniform(math.log(1e-3), math.log(1e-1), size=(E,))
     A = (-np.exp(A_log)).astype(np.float32)
     D = np.ones((E,), dtype=np.float32)
-    return LayerWeights(W_in, W_dt_down, W_B, W_C, W_dt_up, W_out, A, D,
-                        dt_bias.astype(np.float32))
+    lw = LayerWeights(W_in, W_dt_down, W_B, W_C, W_dt_up, W_out, A, D,
+                      dt_bias.astype(np.float32))
+    if wl.block:
+        K = wl.d_conv
+        bound = 1.0 / math.sqrt(K)
+        lw.W_z = w(E, d)
+        lw.conv_w = rng.uniform(-bound, bound, size=(E, K)).astype(np.float32)
+        lw.conv_b = rng.uniform(-bound, bound, size=(E,)).astype(np.float32)
+    return lw
 
 
 def make_inputs(wl: Workload, seed: int = 0, batch: int | None = None,
