@@ -132,16 +132,19 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- byte counts
 
-def scan_bytes_per_token(E, N, R_pad, a16=False, predelta=False):
+def scan_bytes_per_token(E, N, R_pad, a16=False, predelta=False, u_f32=False):
     """Algorithmic HBM bytes of the scan kernel per token.
-    A8 (Delta-up fused): read u (int16 accumulators + one fp32 scale), the
-    Delta-down codes and their factor, B and C (fp32); write y (fp32).
+    A8 (Delta-up fused): read u (int16 accumulators + one fp32 scale; fp32
+    in the six-kernel and block forms), the Delta-down codes and their
+    factor, B and C (fp32); write y (fp32).
     A8 with delta formed before the scan: delta (fp32) instead of the codes.
     A16: read u (bf16), delta (fp32), B and C; write y (bf16)."""
     if a16:
         return E * 2 + E * 4 + 2 * N * 4 + E * 2
     if predelta:
         return E * 2 + 4 + E * 4 + 2 * N * 4 + E * 4
+    if u_f32:
+        return E * 4 + R_pad + 4 + 2 * N * 4 + E * 4
     return E * 2 + 4 + R_pad + 4 + 2 * N * 4 + E * 4
 
 
@@ -173,6 +176,16 @@ def layer_bytes_per_token(wl):
         rms_y = E * 2
         out_proj = E * 2 + d * 2
         return rms_x + in_proj + x_proj + dt_proj + scan_bytes_per_token(E, N, Rp, True) + rms_y + out_proj
+    if wl.block:
+        io = 2 if wl.io_dtype == "bf16" else 4
+        quant_x = d * io + d + 4
+        branches = 2 * (d + 4 + E * 4)          # in_proj and z_proj: read q_x, write fp32
+        conv = E * 4 + E * 4 + E + 4            # read u_pre, write u, q_u, deq_u
+        x_proj = E + 4 + 2 * N * 4 + Rp + 4
+        gate = 2 * E * 4 + E + 4                # read y, z; write q_y, deq_y
+        out_proj = E + 4 + d * io
+        return (quant_x + branches + conv + x_proj + scan_bytes_per_token(E, N, Rp, u_f32=True)
+                + gate + out_proj)
     return pre_bytes_per_token(wl) + scan_bytes_per_token(E, N, Rp) + post_bytes_per_token(wl)
 
 
@@ -426,6 +439,10 @@ def run_ours(args):
     elif act == abi.A8 and nl == 4:
         names = ["expand_weights", "bitssm_pre(quant_x+in_proj+x_proj)",
                  "gemm_dt_proj(+softplus)", "selective_scan", "bitssm_post(quant_y+out_proj)"]
+    elif act == abi.A8 and wl.block:
+        names = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_z_proj",
+                 "conv_silu_quant_u", "gemm_x_proj", "selective_scan_fused_dt",
+                 "gate_quant_y", "gemm_out_proj"]
     elif act == abi.A8:
         names = ["expand_weights", "quant_rows_x", "gemm_in_proj", "gemm_x_proj",
                  "selective_scan_fused_dt", "quant_rows_y", "gemm_out_proj"]
@@ -449,7 +466,8 @@ def run_ours(args):
         achieved = exps / t_s / 1e12
         peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e12
         hbm_bytes = T * scan_bytes_per_token(wl.d_inner, wl.d_state, Rp, act == abi.A16,
-                                             act == abi.A8 and nl == 4)
+                                             act == abi.A8 and nl == 4,
+                                             u_f32=act == abi.A8 and nl > 4)
         roof = {"kernel": names[dom], "bound": "alu", "unit": "Tex2/s",
                 "achieved": round(achieved, 4), "peak": round(peak, 4),
                 "frac": round(achieved / peak, 4),
@@ -492,6 +510,8 @@ def run_ours(args):
                    "parallelism": f"replica x{world}" if world > 1 else "single",
                    "mode": "decode: bitssm_step, one token per sequence, state carried"
                            if decode else "forward over whole sequences",
+                   "block": "Mamba-1 block form: conv1d + SiLU on u, SiLU(z) gate"
+                            if wl.block else None,
                    "l2": "flushed before every timed step (256 MiB write, outside the events)"},
         "roofline": roof,
         "kernel_share": share,

@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define BITSSM_ABI_VERSION 1
+#define BITSSM_ABI_VERSION 2
 
 enum bitssm_status_code {
   BITSSM_OK = 0,
@@ -90,6 +90,18 @@ typedef struct bitssm_tw {
  * store the int8 activation codes of x, u and y in its workspace (see
  * bitssm_workspace_layout; for stage-by-stage checks). */
 #define BITSSM_KEEP_CODES 1
+/* Mamba-1 block form (d_conv != 0; A8 only, from a zero state): the layer
+ * additionally has a gate branch and a depthwise causal conv on u,
+ *   u_pre = BitLinear(x; in_proj),  z = BitLinear(x; z_proj)  (one set of
+ *           int8 codes of x feeds both; z_proj [E, d], its own scale),
+ *   u     = SiLU(conv_b[e] + sum_k conv_w[e, k] * u_pre[t - (d_conv-1) + k, e])
+ *           (left zero padding: tap d_conv-1 is the current step),
+ *   x_proj, Delta, scan as in the mixer, on u (its codes from its float
+ *   value), then y_g = y * SiLU(z) and out = BitLinear(y_g; out_proj).
+ * None of the pages names these pieces; they are the parts of the Mamba-1
+ * block around the same selective scan.  conv_w: float [E, d_conv] (device),
+ * conv_b: float [E] (device) or NULL for zero bias, 1 <= d_conv <= 4.  With
+ * d_conv == 0 the fields z_proj, conv_w and conv_b are ignored. */
 typedef struct bitssm_layer {
   bitssm_tw in_proj, dt_down, b_proj, c_proj, dt_up, out_proj;
   const float* A;
@@ -101,6 +113,10 @@ typedef struct bitssm_layer {
   int dt_rank;
   const void* prepared;
   int flags;
+  bitssm_tw z_proj;
+  const float* conv_w;
+  const float* conv_b;
+  int d_conv;
 } bitssm_layer;
 
 /* Version of this ABI (BITSSM_ABI_VERSION). */
@@ -248,8 +264,10 @@ int bitssm_forward(const bitssm_layer* p, const void* x, void* out, const void* 
  * count): pre, Delta-up + softplus as an int8 GEMM writing delta, the scan
  * reading it, post.  Other A8 shapes: 6 (quantise x, in_proj, x_proj, scan,
  * quantise y, out_proj).  A16: 7 (RMS of x, in_proj, x_proj, dt_proj, scan,
- * RMS of y, out_proj).  Plus 1 (first) for the weight expansion when
- * `prepared` is NULL. */
+ * RMS of y, out_proj).  A8 block form (d_conv != 0): 8 (quantise x,
+ * in_proj, z_proj, conv + SiLU + quantise u, x_proj, scan, gate + quantise
+ * y, out_proj).  Plus 1 (first) for the weight expansion when `prepared`
+ * is NULL. */
 int bitssm_forward_launches(const bitssm_layer* p, int B, int L, int act_mode);
 
 /* bitssm_forward, additionally recording events[i] (cudaEvent_t handles
@@ -271,7 +289,9 @@ int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const 
  * results of one call over the whole sequence.  Arguments otherwise as
  * bitssm_forward (same workspace size for the same B and L); h must not
  * alias x, out or the workspace.  Errors as bitssm_forward; a NULL h is
- * BITSSM_ERR_INVALID_ARG.
+ * BITSSM_ERR_INVALID_ARG; a block-form layer (d_conv != 0, whose conv would
+ * also need the last d_conv - 1 inputs carried) is
+ * BITSSM_ERR_UNSUPPORTED_SHAPE.
  * bitssm_step is the decode step: L = 1, x and out [B, d_model].
  * --------------------------------------------------------------------- */
 int bitssm_forward_state(const bitssm_layer* p, const void* x, void* out, const void* residual,
@@ -338,7 +358,10 @@ int bitssm_prepare_weights(const bitssm_layer* p, int act_mode, void* dst, size_
  *        Cm float [T, N], q_dt int8 [T, ld_qdt], deq_dt float [T],
  *        y float [T, E], q_y int8 [T, ld_qu], deq_y float [T]; delta float
  *        [T, E] only when the forward forms it by a GEMM before the scan
- *        (see bitssm_forward_launches)
+ *        (see bitssm_forward_launches); block form only: u_pre float
+ *        [T, E] (in_proj output before the conv; u then holds the float u
+ *        after conv + SiLU), z float [T, E] (the gate branch); y is the scan
+ *        output before the gate
  *   A16: r_x float [T], u bf16 [T, E], dt_low bf16 [T, R], r_dt float [T],
  *        Bm, Cm float [T, N], delta float [T, E] (= softplus(delta_raw +
  *        dt_bias), formed in the dt_proj epilogue), y bf16 [T, E],
@@ -349,6 +372,7 @@ typedef struct bitssm_ws_view {
   size_t q_x, deq_x, u, q_u, deq_u, Bm, Cm, q_dt, deq_dt, y, q_y, deq_y;
   size_t r_x, dt_low, r_dt, delta_raw, r_y;
   size_t u_scale, delta;
+  size_t u_pre, z;
   int ld_qx, ld_qu, ld_qdt;
   int u_dtype;
 } bitssm_ws_view;

@@ -63,13 +63,14 @@ class bitssm_layer(ctypes.Structure):
                 ("c_proj", bitssm_tw), ("dt_up", bitssm_tw), ("out_proj", bitssm_tw),
                 ("A", _vp), ("D", _vp), ("dt_bias", _vp),
                 ("d_model", _i), ("d_inner", _i), ("d_state", _i), ("dt_rank", _i),
-                ("prepared", _vp), ("flags", _i)]
+                ("prepared", _vp), ("flags", _i),
+                ("z_proj", bitssm_tw), ("conv_w", _vp), ("conv_b", _vp), ("d_conv", _i)]
 
 
 class bitssm_ws_view(ctypes.Structure):
     _fields_ = [(n, _sz) for n in ("q_x", "deq_x", "u", "q_u", "deq_u", "Bm", "Cm", "q_dt",
                                    "deq_dt", "y", "q_y", "deq_y", "r_x", "dt_low", "r_dt",
-                                   "delta_raw", "r_y", "u_scale", "delta")] + \
+                                   "delta_raw", "r_y", "u_scale", "delta", "u_pre", "z")] + \
                [("ld_qx", _i), ("ld_qu", _i), ("ld_qdt", _i), ("u_dtype", _i)]
 
 

@@ -383,8 +383,9 @@ struct LayerPlan {
   int ld_d, ld_E, ld_R;    // padded K pitches (elements)
   int xrows;               // R + 2N
   bool a16;
+  bool block;              // Mamba-1 block form (conv + SiLU on u, SiLU(z) gate)
   // expanded weights (offsets relative to the expanded block)
-  size_t w_in, w_x, w_up, w_out, w_bytes;
+  size_t w_in, w_x, w_up, w_out, w_z, w_bytes;
   // A16: transposed fp32 group scales inside the expanded block
   size_t s_in, s_x, s_up, s_out;
   // workspace offsets (absolute; expanded block at 0 when not prepared)
@@ -413,11 +414,17 @@ bool layer_shape_ok(const bitssm_layer* p, int act_mode) {
   const int want_group = act_mode == BITSSM_A16 ? -1 : 0;
   for (auto w : ws)
     if (want_group == 0 && w->group != 0) return false;
+  if (p->d_conv != 0) {  // Mamba-1 block form
+    if (p->d_conv < 1 || p->d_conv > 4 || p->conv_w == nullptr || !tw_ok(&p->z_proj)) return false;
+    if (p->z_proj.n_out != E || p->z_proj.k_in != d) return false;
+    if (want_group == 0 && p->z_proj.group != 0) return false;
+  }
   return true;
 }
 
 int layer_supported(const bitssm_layer* p, int act_mode) {
   if (p->d_state != kScanN) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (p->d_conv != 0 && act_mode != BITSSM_A8) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (p->d_model % 16 != 0 || p->d_inner % 16 != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   if (act_mode == BITSSM_A8) {
     if (p->d_inner > 512) return BITSSM_ERR_UNSUPPORTED_SHAPE;   // whole u row in one tile
@@ -432,7 +439,7 @@ int layer_supported(const bitssm_layer* p, int act_mode) {
 
 // The A8 layer runs as the fused three-kernel path for these shapes.
 bool a8_fused(const LayerPlan& P) {
-  return (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64 && P.R <= 64;
+  return !P.block && (P.d == 128 || P.d == 256) && (P.E == 256 || P.E == 512) && P.xrows <= 64 && P.R <= 64;
 }
 
 // Fused A8 with few channels (B * E below ~96 per SM sub-partition, where the
@@ -453,6 +460,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   P.N = p->d_state;
   P.R = p->dt_rank;
   P.a16 = act_mode == BITSSM_A16;
+  P.block = p->d_conv != 0;
   P.ld_d = round_up(P.d, 16);
   P.ld_E = round_up(P.E, 16);
   P.ld_R = round_up(P.R, 16);
@@ -463,6 +471,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   P.w_x = o; o = align_up(o + (size_t)P.xrows * P.ld_E * es);
   P.w_up = o; o = align_up(o + (size_t)P.E * P.ld_R * es);
   P.w_out = o; o = align_up(o + (size_t)P.d * P.ld_E * es);
+  if (P.block) { P.w_z = o; o = align_up(o + (size_t)P.E * P.ld_d * es); }
   if (P.a16) {
     P.s_in = o; o = align_up(o + (size_t)scale_groups(P.d) * scale_ld(P.E) * 4);
     P.s_x = o; o = align_up(o + (size_t)scale_groups(P.E) * scale_ld(P.xrows) * 4);
@@ -477,6 +486,7 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
   v.q_x = v.deq_x = v.u = v.q_u = v.deq_u = v.Bm = v.Cm = v.q_dt = v.deq_dt = v.y = v.q_y = v.deq_y = none;
   v.r_x = v.dt_low = v.r_dt = v.delta_raw = v.r_y = none;
   v.u_scale = v.delta = none;
+  v.u_pre = v.z = none;
   v.u_dtype = P.a16 ? BITSSM_BF16 : BITSSM_F32;
   P.ss_u = none;
   auto take = [&](size_t bytes) {
@@ -501,6 +511,10 @@ LayerPlan plan_layer(const bitssm_layer* p, int B, int L, int act_mode, bool pre
     v.y = take(T * P.E * 4);
     v.q_y = take(T * P.ld_E);
     v.deq_y = take(T * 4);
+    if (P.block) {
+      v.u_pre = take(T * P.E * 4);
+      v.z = take(T * P.E * 4);
+    }
   } else {
     P.ss_parts = rowss_parts(P.E);
     v.r_x = take(T * 4);
@@ -540,6 +554,10 @@ void fill_expand_jobs(const bitssm_layer* p, const LayerPlan& P, uint8_t* wbase,
   job(4, p->dt_up, 0, P.w_up, P.ld_R, P.s_up, scale_ld(P.E));
   job(5, p->out_proj, 0, P.w_out, P.ld_E, P.s_out, scale_ld(P.d));
   J.count = 6;
+  if (P.block) {
+    job(6, p->z_proj, 0, P.w_z, P.ld_d, 0, 0);
+    J.count = 7;
+  }
 }
 
 // Expansion of a layer's weights into `wbase` (A16: the padding rows of the
@@ -729,6 +747,28 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
   mk.mark();
   rc = launch_quant_rows(x, dtype, T, P.d, P.d, at<int8_t>(ws, v.q_x), P.ld_d, at<float>(ws, v.deq_x), st);
   if (rc) return rc;
+  if (P.block) {
+    // Mamba-1 block form: the two in_proj branches on the same codes of x,
+    // then u = SiLU(causal conv(u_pre)) and its codes
+    for (int branch = 0; branch < 2; ++branch) {
+      mk.mark();
+      GemmParams G;
+      std::memset(&G, 0, sizeof(G));
+      G.M = T; G.N = P.E; G.K = P.d;
+      G.out_dtype = BITSSM_F32;
+      G.alpha = branch == 0 ? p->in_proj.scales : p->z_proj.scales;
+      G.row_scale = at<float>(ws, v.deq_x);
+      G.out = at<float>(ws, branch == 0 ? v.u_pre : v.z); G.ld_out = P.E;
+      rc = launch_gemm<EPI_STORE>(at<int8_t>(ws, v.q_x), P.ld_d, wexp + (branch == 0 ? P.w_in : P.w_z),
+                                  P.ld_d, P.E, G, st);
+      if (rc) return rc;
+    }
+    mk.mark();
+    conv_silu_quant_kernel<<<rows_grid(T), 256, 0, st>>>(
+        at<float>(ws, v.u_pre), T, L, P.E, p->conv_w, p->conv_b, p->d_conv, at<float>(ws, v.u),
+        at<int8_t>(ws, v.q_u), P.ld_E, at<float>(ws, v.deq_u));
+    if ((rc = launch_status())) return rc;
+  } else {
   // a2 + a3: in_proj, u = acc * s_in * deq_x, codes of u from the int32 row
   mk.mark();
   {
@@ -742,6 +782,7 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     G.deq_out = at<float>(ws, v.deq_u);
     rc = launch_gemm<EPI_QUANT_ROW>(at<int8_t>(ws, v.q_x), P.ld_d, wexp + P.w_in, P.ld_d, P.E, G, st);
     if (rc) return rc;
+  }
   }
   // a4: x_proj (Delta-down | B | C), dt codes from the int32 row
   mk.mark();
@@ -777,10 +818,18 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
     rc = launch_scan<true, float, float, float>(S, st);
     if (rc) return rc;
   }
-  // a7: codes of y
+  // a7: codes of y (block form: of the gated y * SiLU(z))
   mk.mark();
-  rc = launch_quant_rows(at<float>(ws, v.y), BITSSM_F32, T, P.E, P.E, at<int8_t>(ws, v.q_y), P.ld_E,
-                         at<float>(ws, v.deq_y), st);
+  if (P.block) {
+    gate_quant_kernel<<<rows_grid(T), 256, 0, st>>>(at<float>(ws, v.y), at<float>(ws, v.z), T, P.E,
+                                                    at<int8_t>(ws, v.q_y), P.ld_E,
+                                                    at<float>(ws, v.deq_y),
+                                                    (p->flags & BITSSM_KEEP_CODES) ? 1 : 0);
+    rc = launch_status();
+  } else {
+    rc = launch_quant_rows(at<float>(ws, v.y), BITSSM_F32, T, P.E, P.E, at<int8_t>(ws, v.q_y), P.ld_E,
+                           at<float>(ws, v.deq_y), st);
+  }
   if (rc) return rc;
   // a8: out_proj (+ residual)
   mk.mark();
@@ -1160,6 +1209,7 @@ int forward_impl(const bitssm_layer* p, const void* x, void* out, const void* re
                  Marks& mk, float* h = nullptr) {
   int rc = check_layer_args(p, B, L, dtype, act_mode);
   if (rc) return rc;
+  if (h != nullptr && p->d_conv != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
   const long T = (long)B * L;
   if (T > 0 && (x == nullptr || out == nullptr)) return BITSSM_ERR_INVALID_ARG;
   const bool prepared = p->prepared != nullptr;
@@ -1217,6 +1267,7 @@ int bitssm_forward_launches(const bitssm_layer* p, int B, int L, int act_mode) {
   const int expand = p->prepared != nullptr ? 0 : 1;
   if (act_mode == BITSSM_A16) return expand + 7;
   const LayerPlan P = plan_layer(p, B, L, act_mode, p->prepared != nullptr);
+  if (P.block) return expand + 8;
   return expand + (a8_fused(P) ? (P.predelta ? 4 : 3) : 6);
 }
 
@@ -1241,7 +1292,7 @@ int bitssm_stack_forward(const bitssm_layer* layers, int n_layers, const void* x
     int rc = check_layer_args(&layers[l], B, L, dtype, act_mode);
     if (rc) return rc;
     if (layers[l].d_model != layers[0].d_model || layers[l].d_inner != layers[0].d_inner ||
-        layers[l].dt_rank != layers[0].dt_rank)
+        layers[l].dt_rank != layers[0].dt_rank || (layers[l].d_conv != 0) != (layers[0].d_conv != 0))
       return BITSSM_ERR_INVALID_ARG;
   }
   for (int l = 0; l < n_layers; ++l) {

@@ -205,6 +205,97 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(const T* __restrict
   }
 }
 
+// ------------------------------------------------------ Mamba-1 block pieces
+// SiLU(v) = v / (1 + e^-v) in float32 with every step IEEE round-to-nearest
+// (no contraction), so that evaluating it twice gives the same bits.  For
+// v -> -inf, e^-v overflows to inf and the quotient is -0; for v -> +inf it
+// is v.
+__device__ __forceinline__ float silu_rn(float v) {
+  return __fdiv_rn(v, __fadd_rn(1.f, expf(-v)));
+}
+
+// Depthwise causal conv + SiLU on the in_proj branch, then the absmax int8
+// codes of the result (the quantiser above).  One warp per token row
+// t = b * L + l of u_pre [M, E] (M = B * L):
+//   u[t, e] = SiLU(cb[e] + sum_k w[e, k] * u_pre[t - (K-1) + k, e]),
+// a tap that reaches before the start of its sequence (l - (K-1) + k < 0)
+// contributes nothing.  w float [E, K], cb float [E] or null (zero).
+// Writes u float [M, E], q int8 [M, ldq] (columns E..ldq-1 zero), deq [M].
+__global__ void __launch_bounds__(256) conv_silu_quant_kernel(
+    const float* __restrict__ u_pre, int M, int L, int E, const float* __restrict__ w,
+    const float* __restrict__ cb, int K, float* __restrict__ u, int8_t* __restrict__ q, long ldq,
+    float* __restrict__ deq) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const int l = (int)(row % L);
+    const int taps = K < l + 1 ? K : l + 1;  // taps inside the sequence
+    float mx = 0.f, ss = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      float acc = cb != nullptr ? __ldg(cb + e) : 0.f;
+      for (int back = 0; back < taps; ++back)  // back = steps into the past
+        acc = fmaf(__ldg(w + (long)e * K + (K - 1 - back)), __ldg(u_pre + (row - back) * E + e), acc);
+      const float v = silu_rn(acc);
+      u[row * E + e] = v;
+      mx = fmaxf(mx, fabsf(v));
+      ss = fmaf(v, v, ss);
+    }
+    mx = warp_max(mx);
+    ss = warp_sum(ss);
+    const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+    int8_t* qr = q + row * ldq;
+    // each lane reads back only the elements it wrote itself
+    for (int e = lane; e < ldq; e += 32)
+      qr[e] = e < E ? (int8_t)quant_code(u[row * E + e], sigma) : (int8_t)0;
+    if (lane == 0) {
+      const float r = 1.0f / sqrtf(ss / (float)E + kEpsNorm);
+      deq[row] = mx * r / 127.f;
+    }
+  }
+}
+
+// The gate of the Mamba-1 block and the absmax codes of the gated row: one
+// warp per row, y_g = y * SiLU(z) (y, z float [M, E]), then q int8 [M, ldq]
+// and deq [M] of y_g as quant_rows_kernel.  y_g is formed twice (for the row
+// statistics, then for the codes), bit-identically.  With keep != 0, y is
+// overwritten with y_g (for stage checks).
+__global__ void __launch_bounds__(256) gate_quant_kernel(float* __restrict__ y,
+                                                         const float* __restrict__ z, int M, int E,
+                                                         int8_t* __restrict__ q, long ldq,
+                                                         float* __restrict__ deq, int keep) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    float* yr = y + row * E;
+    const float* zr = z + row * E;
+    float mx = 0.f, ss = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      const float g = __fmul_rn(yr[e], silu_rn(__ldg(zr + e)));
+      mx = fmaxf(mx, fabsf(g));
+      ss = fmaf(g, g, ss);
+    }
+    mx = warp_max(mx);
+    ss = warp_sum(ss);
+    const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+    int8_t* qr = q + row * ldq;
+    for (int e = lane; e < ldq; e += 32) {
+      int c = 0;
+      if (e < E) {
+        const float g = __fmul_rn(yr[e], silu_rn(__ldg(zr + e)));
+        c = quant_code(g, sigma);
+        if (keep) yr[e] = g;
+      }
+      qr[e] = (int8_t)c;
+    }
+    if (lane == 0) {
+      const float r = 1.0f / sqrtf(ss / (float)E + kEpsNorm);
+      deq[row] = mx * r / 127.f;
+    }
+  }
+}
+
 // r[m] = 1 / sqrt(mean(x[m]^2) + eps), one warp per row.
 template <typename T>
 __global__ void __launch_bounds__(256) row_rms_kernel(const T* __restrict__ x, int M, int K,

@@ -56,6 +56,14 @@ class DeviceLayer:
             m["W_in"].tw, m["W_dt_down"].tw, m["W_B"].tw, m["W_C"].tw, m["W_dt_up"].tw,
             m["W_out"].tw, self.A.data_ptr(), self.D.data_ptr(), self.dt_bias.data_ptr(),
             lw.W_in.shape[1], lw.W_in.shape[0], lw.A.shape[1], lw.W_dt_down.shape[0], None, 0)
+        if getattr(lw, "W_z", None) is not None:  # Mamba-1 block form
+            self.mats["W_z"] = PackedMatrix(lw.W_z, group, device, stream)
+            self.conv_w = torch.from_numpy(np.ascontiguousarray(lw.conv_w, dtype=np.float32)).to(device)
+            self.conv_b = torch.from_numpy(np.ascontiguousarray(lw.conv_b, dtype=np.float32)).to(device)
+            self.layer.z_proj = self.mats["W_z"].tw
+            self.layer.conv_w = self.conv_w.data_ptr()
+            self.layer.conv_b = self.conv_b.data_ptr()
+            self.layer.d_conv = lw.conv_w.shape[1]
         self._prepared = None
 
     def prepare(self, stream=None):

@@ -45,7 +45,7 @@ def test_binding_names_match_header_and_host_calls():
     ensure_built()
     from ternary_weight_selective_b200 import bitssm as abi
     assert set(abi.EXPORTS) == set(declared_functions())
-    assert abi.bitssm_version() == 1
+    assert abi.bitssm_version() == 2
     assert abi.bitssm_status_string(abi.ERR_WORKSPACE).startswith("workspace")
     # host-only argument checks return statuses without touching a device
     import pytest
