@@ -144,6 +144,15 @@ int launch_gemm(const void* A, long lda, const void* W, long ldw, long w_rows, c
     return launch_gemm_bn<256, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
   }
   const int need = EPI == EPI_STORE ? (P.N < 256 ? P.N : 256) : P.N;
+  if constexpr (EPI == EPI_STORE) {
+    // at most two K panels: two stages, so that two CTAs share an SM and one
+    // CTA's epilogue stores overlap the other's loads
+    if (P.K <= 256) {
+      if (need <= 64) return launch_gemm_bn<64, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+      if (need <= 128) return launch_gemm_bn<128, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+      return launch_gemm_bn<256, EPI, 2>(A, lda, W, ldw, w_rows, P, st);
+    }
+  }
   if (need <= 64) return launch_gemm_bn<64, EPI>(A, lda, W, ldw, w_rows, P, st);
   if (need <= 128) return launch_gemm_bn<128, EPI>(A, lda, W, ldw, w_rows, P, st);
   if (need <= 256) return launch_gemm_bn<256, EPI>(A, lda, W, ldw, w_rows, P, st);
@@ -261,6 +270,58 @@ int launch_quant_rows(const void* x, int dtype, int M, int K, long ldx, int8_t* 
   else
     quant_rows_kernel<__nv_bfloat16><<<rows_grid(M), 256, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(x), M, K, ldx, q, ldq, deq);
+  return launch_status();
+}
+
+// Block-form row kernels: the vector forms for d_inner a multiple of 128 up
+// to 512 (rows of whole 16-byte vectors, one to four per lane), else the
+// scalar forms.
+bool vec_rows_ok(int E, const void* a, const void* b) {
+  return E % 128 == 0 && E <= 512 && (reinterpret_cast<uintptr_t>(a) & 15) == 0 &&
+         (reinterpret_cast<uintptr_t>(b) & 15) == 0;
+}
+
+// Grid of the vector row kernels: about as many 256-thread blocks as fit on
+// the SMs at once, each warp looping over rows (the conv kernel stages its
+// taps in shared memory once per block, so short-lived blocks would repeat
+// that for every eight rows).
+inline int vec_rows_grid(long M, int blocks_per_sm) {
+  const long g = (M + 7) / 8;
+  const long cap = (long)num_sms() * blocks_per_sm;
+  return (int)(g < cap ? (g < 1 ? 1 : g) : cap);
+}
+
+int launch_conv_silu_quant(const float* u_pre, int M, int L, int E, const float* w, const float* cb,
+                           int K, float* u, int8_t* q, long ldq, float* deq, cudaStream_t st) {
+  if (M == 0) return BITSSM_OK;
+  if (vec_rows_ok(E, u_pre, u)) {
+    const int g = vec_rows_grid(M, 3);
+    switch (E / 128) {
+      case 1: conv_silu_quant_vec_kernel<1><<<g, 256, 0, st>>>(u_pre, M, L, E, w, cb, K, u, q, ldq, deq); break;
+      case 2: conv_silu_quant_vec_kernel<2><<<g, 256, 0, st>>>(u_pre, M, L, E, w, cb, K, u, q, ldq, deq); break;
+      case 3: conv_silu_quant_vec_kernel<3><<<g, 256, 0, st>>>(u_pre, M, L, E, w, cb, K, u, q, ldq, deq); break;
+      default: conv_silu_quant_vec_kernel<4><<<g, 256, 0, st>>>(u_pre, M, L, E, w, cb, K, u, q, ldq, deq); break;
+    }
+  } else {
+    conv_silu_quant_kernel<<<rows_grid(M), 256, 0, st>>>(u_pre, M, L, E, w, cb, K, u, q, ldq, deq);
+  }
+  return launch_status();
+}
+
+int launch_gate_quant(float* y, const float* z, int M, int E, int8_t* q, long ldq, float* deq,
+                      int keep, cudaStream_t st) {
+  if (M == 0) return BITSSM_OK;
+  if (vec_rows_ok(E, y, z)) {
+    const int g = vec_rows_grid(M, 4);
+    switch (E / 128) {
+      case 1: gate_quant_vec_kernel<1><<<g, 256, 0, st>>>(y, z, M, E, q, ldq, deq, keep); break;
+      case 2: gate_quant_vec_kernel<2><<<g, 256, 0, st>>>(y, z, M, E, q, ldq, deq, keep); break;
+      case 3: gate_quant_vec_kernel<3><<<g, 256, 0, st>>>(y, z, M, E, q, ldq, deq, keep); break;
+      default: gate_quant_vec_kernel<4><<<g, 256, 0, st>>>(y, z, M, E, q, ldq, deq, keep); break;
+    }
+  } else {
+    gate_quant_kernel<<<rows_grid(M), 256, 0, st>>>(y, z, M, E, q, ldq, deq, keep);
+  }
   return launch_status();
 }
 
@@ -764,10 +825,10 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
       if (rc) return rc;
     }
     mk.mark();
-    conv_silu_quant_kernel<<<rows_grid(T), 256, 0, st>>>(
-        at<float>(ws, v.u_pre), T, L, P.E, p->conv_w, p->conv_b, p->d_conv, at<float>(ws, v.u),
-        at<int8_t>(ws, v.q_u), P.ld_E, at<float>(ws, v.deq_u));
-    if ((rc = launch_status())) return rc;
+    rc = launch_conv_silu_quant(at<float>(ws, v.u_pre), T, L, P.E, p->conv_w, p->conv_b, p->d_conv,
+                                at<float>(ws, v.u), at<int8_t>(ws, v.q_u), P.ld_E,
+                                at<float>(ws, v.deq_u), st);
+    if (rc) return rc;
   } else {
   // a2 + a3: in_proj, u = acc * s_in * deq_x, codes of u from the int32 row
   mk.mark();
@@ -821,11 +882,8 @@ int forward_a8(const bitssm_layer* p, const LayerPlan& P, const uint8_t* wexp, c
   // a7: codes of y (block form: of the gated y * SiLU(z))
   mk.mark();
   if (P.block) {
-    gate_quant_kernel<<<rows_grid(T), 256, 0, st>>>(at<float>(ws, v.y), at<float>(ws, v.z), T, P.E,
-                                                    at<int8_t>(ws, v.q_y), P.ld_E,
-                                                    at<float>(ws, v.deq_y),
-                                                    (p->flags & BITSSM_KEEP_CODES) ? 1 : 0);
-    rc = launch_status();
+    rc = launch_gate_quant(at<float>(ws, v.y), at<float>(ws, v.z), T, P.E, at<int8_t>(ws, v.q_y),
+                           P.ld_E, at<float>(ws, v.deq_y), (p->flags & BITSSM_KEEP_CODES) ? 1 : 0, st);
   } else {
     rc = launch_quant_rows(at<float>(ws, v.y), BITSSM_F32, T, P.E, P.E, at<int8_t>(ws, v.q_y), P.ld_E,
                            at<float>(ws, v.deq_y), st);

@@ -348,28 +348,37 @@ __global__ void __launch_bounds__(GemmConfig<BN, STAGES, CSPLIT>::kThreads, 1)
 
     if constexpr (EPI == EPI_STORE) {
       const float f = (P.alpha != nullptr ? *P.alpha : 1.f) * rs;
-      const int ncols = min(BN, P.N - n0);
+      if (P.out_dtype == 2) {
+        // raw int32 accumulators (bit-exact checks): straight from each lane's row
+        const int ncols = min(BN, P.N - n0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(trow + c0, r);
-        if (!ok || !live) continue;
+        for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(trow + c0, r);
+          if (!ok || !live) continue;
+          const int col = cs + c0;
+          const int valid = min(32, ncols - col);
+          int* o = reinterpret_cast<int*>(P.out) + (long)m * P.ld_out + n0 + col;
+          for (int j = 0; j < valid; ++j) o[j] = (int)r[j];
+        }
+      } else {
+        // f32 / bf16: 32 x 32 blocks transposed through per-warp buffers in
+        // the idle pipeline stages, so that every store is a coalesced row
+        // segment (rows >= M and columns >= N are skipped inside)
+        static_assert(4 * CSPLIT * kStageFloats * 4 <= STAGES * Cfg::kStageBytes, "output staging");
+        float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * kStageFloats;
+#pragma unroll 1
+        for (int c0 = 0; c0 < Cfg::kSlice; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(trow + c0, r);
+          float v[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int col = cs + c0 + hh * 16;
-          if (col >= ncols) break;
-          const int valid = min(16, ncols - col);
-          const long idx = (long)m * P.ld_out + n0 + col;
-          if (P.out_dtype == 2) {
-            int* o = reinterpret_cast<int*>(P.out) + idx;
-            for (int j = 0; j < valid; ++j) o[j] = (int)r[hh * 16 + j];
-            continue;
-          }
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = i2f_exact((int)r[hh * 16 + j]) * f;
-          if (P.residual != nullptr) add_residual16(P.residual, idx, P.out_dtype, v, valid);
-          store16(P.out, idx, P.out_dtype, v, valid);
+          for (int j = 0; j < 32; ++j) v[j] = i2f_exact((int)r[j]) * f;
+          if (!ok) continue;
+          if (P.out_dtype == 1)
+            warp_store_block<1>(stg, v, lane, P.out, P.residual, P.ld_out, m0 + q * 32, n0 + cs + c0, P.M, P.N);
+          else
+            warp_store_block<0>(stg, v, lane, P.out, P.residual, P.ld_out, m0 + q * 32, n0 + cs + c0, P.M, P.N);
         }
       }
     } else if constexpr (EPI == EPI_DELTA) {

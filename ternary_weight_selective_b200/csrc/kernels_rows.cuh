@@ -296,6 +296,133 @@ __global__ void __launch_bounds__(256) gate_quant_kernel(float* __restrict__ y,
   }
 }
 
+// SiLU on the special-function unit: v * 1 / (1 + 2^(-v log2 e)), with the
+// IEEE-rounded reciprocal.  Relative error about |v| * 6e-8 + 3e-7 (the
+// exp2 approximation and the rounding of its argument); -0 for v -> -inf.
+__device__ __forceinline__ float silu_fast(float v) {
+  return v * __frcp_rn(1.f + ex2_approx(-v * kLog2e));
+}
+
+__device__ __forceinline__ float4 silu4(float4 a) {
+  return make_float4(silu_fast(a.x), silu_fast(a.y), silu_fast(a.z), silu_fast(a.w));
+}
+
+// Row statistics and codes of VPL float4 vectors per lane (the quantiser
+// above); every lane of the warp calls it for one row.
+template <int VPL>
+__device__ __forceinline__ void quant_row_regs(const float4 (&v)[VPL], int lane, int E,
+                                               int8_t* qr, long ldq, float* deq_row) {
+  float mx = 0.f, ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    ss = fmaf(v[i].x, v[i].x, ss);
+    ss = fmaf(v[i].y, v[i].y, ss);
+    ss = fmaf(v[i].z, v[i].z, ss);
+    ss = fmaf(v[i].w, v[i].w, ss);
+  }
+  mx = warp_max(mx);
+  ss = warp_sum(ss);
+  const float sigma = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    *reinterpret_cast<uint32_t*>(qr + (i * 32 + lane) * 4) =
+        pack4(code_bits(v[i].x, sigma), code_bits(v[i].y, sigma), code_bits(v[i].z, sigma),
+              code_bits(v[i].w, sigma));
+  for (long k = (long)VPL * 128 + lane; k < ldq; k += 32) qr[k] = 0;
+  if (lane == 0) {
+    const float r = 1.0f / sqrtf(ss / (float)E + kEpsNorm);
+    *deq_row = mx * r / 127.f;
+  }
+}
+
+// Vector form of conv_silu_quant_kernel for E = 128 * VPL: each lane holds
+// 4 * VPL channels of its row in registers (16-byte loads of all the taps'
+// rows at once, coalesced across the warp), the taps are staged transposed
+// ([tap][channel]) in shared memory, and the codes are written as one word
+// per 4 channels.  u_pre and u 16-byte aligned.
+template <int VPL>
+__global__ void __launch_bounds__(256) conv_silu_quant_vec_kernel(
+    const float* __restrict__ u_pre, int M, int L, int E, const float* __restrict__ w,
+    const float* __restrict__ cb, int K, float* __restrict__ u, int8_t* __restrict__ q, long ldq,
+    float* __restrict__ deq) {
+  __shared__ float4 s_w[4][VPL * 32];
+  __shared__ float4 s_b[VPL * 32];
+  for (int i = threadIdx.x; i < VPL * 32; i += blockDim.x) {
+    const int c = 4 * i;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      s_w[k][i] = k < K ? make_float4(__ldg(w + (long)c * K + k), __ldg(w + (long)(c + 1) * K + k),
+                                      __ldg(w + (long)(c + 2) * K + k), __ldg(w + (long)(c + 3) * K + k))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    s_b[i] = cb != nullptr ? make_float4(__ldg(cb + c), __ldg(cb + c + 1), __ldg(cb + c + 2), __ldg(cb + c + 3))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    const int l = (int)(row % L);
+    float4 tap[4][VPL];
+#pragma unroll
+    for (int back = 0; back < 4; ++back)  // back = steps into the past
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        tap[back][i] = (back < K && back <= l)
+                           ? __ldg(reinterpret_cast<const float4*>(u_pre + (row - back) * E) + i * 32 + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      float4 a = s_b[i * 32 + lane];
+#pragma unroll
+      for (int back = 0; back < 4; ++back) {
+        if (back < K) {
+          const float4 t = s_w[K - 1 - back][i * 32 + lane];
+          a.x = fmaf(t.x, tap[back][i].x, a.x);
+          a.y = fmaf(t.y, tap[back][i].y, a.y);
+          a.z = fmaf(t.z, tap[back][i].z, a.z);
+          a.w = fmaf(t.w, tap[back][i].w, a.w);
+        }
+      }
+      v[i] = silu4(a);
+      reinterpret_cast<float4*>(u + row * E)[i * 32 + lane] = v[i];
+    }
+    quant_row_regs<VPL>(v, lane, E, q + row * ldq, ldq, deq + row);
+  }
+}
+
+// Vector form of gate_quant_kernel for E = 128 * VPL: y_g = y * SiLU(z)
+// formed once in registers; y and z 16-byte aligned.
+template <int VPL>
+__global__ void __launch_bounds__(256) gate_quant_vec_kernel(float* __restrict__ y,
+                                                             const float* __restrict__ z, int M,
+                                                             int E, int8_t* __restrict__ q,
+                                                             long ldq, float* __restrict__ deq,
+                                                             int keep) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long row = (long)blockIdx.x * warps + (threadIdx.x >> 5); row < M;
+       row += (long)gridDim.x * warps) {
+    float4* yr = reinterpret_cast<float4*>(y + row * E);
+    const float4* zr = reinterpret_cast<const float4*>(z + row * E);
+    float4 yv[VPL], zv[VPL], g[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      yv[i] = yr[i * 32 + lane];
+      zv[i] = __ldg(zr + i * 32 + lane);
+    }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const float4 sz = silu4(zv[i]);
+      g[i] = make_float4(yv[i].x * sz.x, yv[i].y * sz.y, yv[i].z * sz.z, yv[i].w * sz.w);
+      if (keep) yr[i * 32 + lane] = g[i];
+    }
+    quant_row_regs<VPL>(g, lane, E, q + row * ldq, ldq, deq + row);
+  }
+}
+
 // r[m] = 1 / sqrt(mean(x[m]^2) + eps), one warp per row.
 template <typename T>
 __global__ void __launch_bounds__(256) row_rms_kernel(const T* __restrict__ x, int M, int K,
