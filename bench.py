@@ -614,6 +614,176 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+# ---------------------------------------------------------------- SSD scan
+
+SSD_WORKLOADS = {
+    # Mamba-2 1.3B's scan: 64 heads of 64 channels (d_inner 4096), N = 128,
+    # one B/C group; 4 sequences of 2048 tokens
+    "ssd_mamba2_1p3b": dict(B=4, L=2048, H=64, P=64, G=1, N=128),
+}
+SSD_METRIC = "SSD scan (Mamba-2, one decay per head) tokens/s on 1 B200; % of the fp32 FMA roofline"
+
+
+def ssd_oracle_rate(cfg, budget_s):
+    """The oracle's step-by-step SSD on whole sequences of the workload's
+    length, repeated until ~budget_s of CPU work; returns (tokens/s, sample)."""
+    from oracle import ssd_oracle as SSD
+    from ternary_weight_selective_b200 import synthetic as S
+    c = cfg
+    args_ = S.random_ssd_inputs(1, 1, c["L"], c["H"], c["P"], c["G"], c["N"])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        SSD.ssd_sequential(*args_)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return n * c["L"] / el, f"{n} x (1 sequence x {c['L']} tokens), step-by-step float64 recurrence"
+
+
+def run_ssd(args):
+    cfg = SSD_WORKLOADS[args.workload]
+    Bsz, L, H, P, G, N = (cfg[k] for k in ("B", "L", "H", "P", "G", "N"))
+    T = Bsz * L
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        rate, sample = ssd_oracle_rate(cfg, args.cpu_seconds)
+        print(json.dumps({
+            "metric": SSD_METRIC, "value": round(rate, 1), "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(T / rate * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, **cfg, "parallelism": "cpu"},
+            "cpu_baseline": {"value": round(rate, 1), "unit": UNIT, "cores": _oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(rate, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+    import torch
+
+    from ternary_weight_selective_b200 import bitssm as abi
+    from ternary_weight_selective_b200 import synthetic as S
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    host = [torch.from_numpy(a) for a in S.random_ssd_inputs(0, Bsz, L, H, P, G, N)]
+    xd, dtd, Ad, Bd, Cd, Dd = [h.cuda() for h in host]
+    y = torch.empty((Bsz, L, H, P), dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step(st=None):
+        abi.ssd_scan_forward(xd, dtd, Ad, Bd, Cd, Dd, None, y, None, Bsz, L, H, P, G, N,
+                             st if st is not None else torch.cuda.current_stream())
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    Gr = max(1, min(args.steps, 50))
+    R = (args.steps + Gr - 1) // Gr
+
+    def capture(with_step):
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cap):
+            for _ in range(Gr):
+                flush.zero_()
+                if with_step:
+                    step(cap)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    g_plain, g_flush = capture(True), capture(False)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def replay_ms(g):
+        ea.record()
+        g.replay()
+        eb.record()
+        torch.cuda.synchronize()
+        return ea.elapsed_time(eb)
+
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    plain = fl = 0.0
+    for _ in range(R):
+        plain += replay_ms(g_plain)
+        fl += replay_ms(g_flush)
+    clocks = sampler.stop()
+    K = Gr * R
+    ms = (plain - fl) / K
+    value = T / (ms / 1e3)
+    # the one kernel's own duration, events around it on its stream
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k_ms = 0.0
+    for _ in range(5):
+        flush.zero_()
+        e0.record(st)
+        step(st)
+        e1.record(st)
+        torch.cuda.synchronize()
+        k_ms += e0.elapsed_time(e1) / 5
+    # end to end: host page-locked inputs in, result out, every step
+    pin = [h.pin_memory() for h in host]
+    y_host = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
+    dev_in = [xd, dtd, Ad, Bd, Cd, Dd]
+
+    def e2e_step():
+        for d_, h_ in zip(dev_in, pin):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = min(K, 20)
+    ea.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    eb.record()
+    torch.cuda.synchronize()
+    e2e_ms = ea.elapsed_time(eb) / n_e2e
+    h2d = sum(h.numel() * 4 for h in host)
+    peaks, peak_kind = load_peaks()
+    sm_max = (clocks or {}).get("sm_max_mhz") or peaks.get("sm_max_mhz", SM_MAX_MHZ)
+    flops = T * H * P * N * 4          # two FMAs per state and step: the update and C . S
+    fma_peak = SM_COUNT * 128 * 2 * sm_max * 1e6 / 1e12
+    achieved = flops / (k_ms / 1e3) / 1e12
+    hbm_bytes = T * (H * P * 4 * 2 + H * 4 + 2 * G * N * 4)
+    line = {
+        "metric": SSD_METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": 1,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, **cfg, "parallelism": "single",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+        "roofline": {"kernel": "ssd_scan_kernel", "bound": "alu", "unit": "TFLOP/s",
+                     "achieved": round(achieved, 3), "peak": round(fma_peak, 2),
+                     "frac": round(achieved / fma_peak, 4),
+                     "peak_source": f"148 SMs x 128 fp32 lanes x 2 flop x {sm_max:.0f} MHz (FMA issue bound)",
+                     "traffic": None, "hbm_achieved_gbs": round(hbm_bytes / (k_ms / 1e3) / 1e9, 1),
+                     "hbm_frac": round(hbm_bytes / (k_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "hbm_peak_source": f"{peak_kind} hbm_gbs"},
+        "kernel_avg_us": round(k_ms * 1e3, 2),
+        "e2e": {"value": round(T / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": y.numel() * 4,
+                "pipelining": "none: copy in, scan, copy out on one stream"},
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        rate, sample = ssd_oracle_rate(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(rate, 1), "unit": UNIT, "cores": _oracle_threads(),
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -626,7 +796,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.workload in SSD_WORKLOADS:
+        run_ssd(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -280,6 +280,30 @@ int bitssm_forward_timed(const bitssm_layer* p, const void* x, void* out, const 
                          void* const* events, int n_events, void* stream);
 
 /* ---------------------------------------------------------------------
+ * SSD scan (Mamba-2): the selective recurrence with one decay per head
+ * ("Ternary Mamba" abstract: the W1.58A16 model is Mamba-2 1.3B; "SSDi8"
+ * abstract: SSD, the state space duality of Mamba-2).  For sequence b, head
+ * h of H with head dimension P, and B/C group g = h / (H / G) of G:
+ *   S_t = exp(dt_t[h] A[h]) S_{t-1} + dt_t[h] x_t[h] (outer) B_t[g]
+ *   y_t[h] = S_t C_t[g] + D[h] x_t[h]            (S: [P, N] per head)
+ * x, y: float [B, L, H, P]; dt: float [B, L, H], the step after its softplus
+ * (> 0); A: float [H] (< 0); Bm, Cm: float [B, L, G, N]; D: float [H] or
+ * NULL (zero); S0: float [B, H, P, N] starting state or NULL (zero);
+ * S_last: float [B, H, P, N] or NULL, receives the state after the last step
+ * (may alias S0: each state is read before it is written, by one thread).
+ * Supported: N = 16 * 2^k up to 512 and P * N / 16 a multiple of 32 up to
+ * 1024 (for example P = 64, N = 128), B <= 65535; otherwise
+ * BITSSM_ERR_UNSUPPORTED_SHAPE.  H % G != 0, a negative size or (with
+ * B > 0) a NULL required pointer: BITSSM_ERR_INVALID_ARG; B = 0 does
+ * nothing.  The exp is the exp2 unit's
+ * approximation of exp2(dt A log2 e) (relative error ~2^-22); the
+ * recurrence is float32.
+ * --------------------------------------------------------------------- */
+int ssd_scan_forward(const float* x, const float* dt, const float* A, const float* Bm,
+                     const float* Cm, const float* D, const float* S0, float* y, float* S_last,
+                     int B, int L, int H, int P, int G, int N, void* stream);
+
+/* ---------------------------------------------------------------------
  * Forward with a carried state: the recurrent form of the same layer
  * ("Ternary Mamba" abstract: SSMs offer linear-time inference; the state h
  * is all that links one step to the next).  h [B, d_inner, d_state] float:

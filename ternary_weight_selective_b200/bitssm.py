@@ -98,6 +98,7 @@ _SIGS = {
                                  _vp]),
     "bitssm_forward_launches": (_i, [_P_LAYER, _i, _i, _i]),
     "bitssm_selftest_wait": (_i, [ctypes.c_uint, _vp]),
+    "ssd_scan_forward": (_i, [_vp] * 9 + [_i] * 6 + [_vp]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
                                   ctypes.POINTER(_vp), _i, _vp]),
     "bitssm_prepared_size": (_i, [_P_LAYER, _i, ctypes.POINTER(_sz)]),
@@ -226,6 +227,12 @@ def bitssm_step(layer: bitssm_layer, x, out, residual, h, B, dtype, act_mode, ws
     _check(_lib.bitssm_step(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual), _ptr(h), B,
                             dtype, act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitssm_step")
+
+
+def ssd_scan_forward(x, dt, A, Bm, Cm, D, S0, y, S_last, B, L, H, P, G, N, stream=None):
+    _check(_lib.ssd_scan_forward(_ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(S0),
+                                 _ptr(y), _ptr(S_last), B, L, H, P, G, N, _stream(stream)),
+           "ssd_scan_forward")
 
 
 def bitssm_selftest_wait(limit_us: int, stream=None):

@@ -17,6 +17,7 @@
 #include "kernel_fused.cuh"
 #include "kernel_gemm.cuh"
 #include "kernel_scan.cuh"
+#include "kernel_ssd.cuh"
 #include "kernels_rows.cuh"
 #include "ptx.cuh"
 
@@ -1211,6 +1212,33 @@ int selective_scan_forward(const void* u, const void* delta_raw, const float* de
   cudaStream_t st = as_stream(stream);
   if (dtype == BITSSM_F32) return launch_scan<false, float, float, float>(S, st);
   return launch_scan<false, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(S, st);
+}
+
+// ---------------------------------------------------------------- SSD scan
+int ssd_scan_forward(const float* x, const float* dt, const float* A, const float* Bm,
+                     const float* Cm, const float* D, const float* S0, float* y, float* S_last,
+                     int B, int L, int H, int P, int G, int N, void* stream) {
+  if (B < 0 || L < 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0 || H % G != 0)
+    return BITSSM_ERR_INVALID_ARG;
+  const int tpp = N / kSsdNS;
+  if (N % kSsdNS != 0 || tpp > 32 || (tpp & (tpp - 1)) != 0) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  const long threads = (long)P * tpp;
+  if (threads % 32 != 0 || threads > 1024 || B > 65535) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return BITSSM_OK;  // nothing to do
+  if (A == nullptr) return BITSSM_ERR_INVALID_ARG;
+  if (L > 0 && (x == nullptr || dt == nullptr || Bm == nullptr || Cm == nullptr || y == nullptr))
+    return BITSSM_ERR_INVALID_ARG;
+  const size_t smem = ssd_smem_bytes(P, N);
+  if (smem > 200 * 1024) return BITSSM_ERR_UNSUPPORTED_SHAPE;
+  if (smem > 48 * 1024) {
+    static std::atomic<uint64_t> attr_done{0};
+    if (int rc = set_smem_attr_once(ssd_scan_kernel, (int)smem, attr_done)) return rc;
+  }
+  SsdParams Q;
+  Q.x = x; Q.dt = dt; Q.A = A; Q.Bm = Bm; Q.Cm = Cm; Q.D = D; Q.S0 = S0; Q.y = y; Q.S_last = S_last;
+  Q.B = B; Q.L = L; Q.H = H; Q.P = P; Q.G = G; Q.N = N;
+  ssd_scan_kernel<<<dim3((unsigned)H, (unsigned)B), (unsigned)threads, smem, as_stream(stream)>>>(Q);
+  return launch_status();
 }
 
 // ---------------------------------------------------------------- layer

@@ -199,3 +199,18 @@ def random_scan_inputs(seed: int, B: int, L: int, E: int, N: int):
     D = np.ones((E,), dtype=np.float32)
     dt_bias = rng.uniform(math.log(1e-3), math.log(1e-1), size=(E,)).astype(np.float32)
     return u, delta_raw, dt_bias, A, Bm, Cm, D
+
+
+def random_ssd_inputs(seed: int, B: int, L: int, H: int, P: int, G: int, N: int):
+    """Inputs of the SSD scan alone, drawn as Mamba-2 initialises them:
+    x, B, C ~ N(0,1); the step dt log-uniform in [1e-3, 1e-1] (the range its
+    dt bias is initialised to give); A = -U(1, 16) per head; D = 1.
+    Returns float32 arrays x [B,L,H,P], dt [B,L,H], A [H], Bm, Cm [B,L,G,N], D [H]."""
+    rng = np.random.default_rng(seed)
+    x = rng.normal(0.0, 1.0, size=(B, L, H, P)).astype(np.float32)
+    dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=(B, L, H))).astype(np.float32)
+    A = (-rng.uniform(1.0, 16.0, size=(H,))).astype(np.float32)
+    Bm = rng.normal(0.0, 1.0, size=(B, L, G, N)).astype(np.float32)
+    Cm = rng.normal(0.0, 1.0, size=(B, L, G, N)).astype(np.float32)
+    D = np.ones((H,), dtype=np.float32)
+    return x, dt, A, Bm, Cm, D
