@@ -1,4 +1,5 @@
-"""CPU oracle for the BitSSM forward pass.
+"""CPU oracle for the BitSSM forward pass: numpy (bitssm_oracle, ssd_oracle)
+and a plain C host oracle (c/, loaded by c_oracle) held to it.
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
 execute anything in this package: only ``tests/``, ``__graft_entry__.smoke()``
