@@ -534,6 +534,9 @@ def run_ours(args):
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+        c_line = cpu_baseline_c(wl, budget_s=min(5.0, args.cpu_seconds))
+        if c_line is not None:
+            line["cpu_baseline"]["c_oracle"] = c_line
     print(json.dumps(line))
 
 
@@ -579,6 +582,32 @@ def cpu_baseline(wl, budget_s: float = 12.0):
     return {"value": round(tokens * n / el, 1), "unit": UNIT, "cores": _oracle_threads(),
             "kind": "oracle", "sample": f"{n} x {seqs} sequences x {wl.seqlen} tokens "
                                         f"({wl.layers} layer(s)), {el:.1f} s"}
+
+
+def cpu_baseline_c(wl, budget_s: float = 5.0):
+    """The C host oracle (oracle/c/, OpenMP over token rows and scan channels,
+    every host core) on the same kind of sample: whole sequences of one layer,
+    repeated until ~budget_s.  None for the workloads it does not cover (the
+    stack, the block form)."""
+    if wl.layers != 1 or getattr(wl, "block", False):
+        return None
+    from oracle import c_oracle as C
+    from ternary_weight_selective_b200 import synthetic as S
+    seqs = max(1, min(wl.batch, 4, 1024 // wl.seqlen))
+    x, layers = S.make_inputs(wl, seed=0, batch=seqs)
+    P = C.Layer(layers[0], wl.act_mode)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        C.bitssm_forward(x, P)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 200:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count() or 1
+    return {"value": round(seqs * wl.seqlen * n / el, 1), "unit": UNIT, "cores": cores,
+            "kind": "oracle (C, OpenMP)",
+            "sample": f"{n} x {seqs} sequences x {wl.seqlen} tokens, {el:.1f} s"}
 
 
 def run_reference(args):
