@@ -537,6 +537,8 @@ def run_ours(args):
         c_line = cpu_baseline_c(wl, budget_s=min(5.0, args.cpu_seconds))
         if c_line is not None:
             line["cpu_baseline"]["c_oracle"] = c_line
+            if wl.name in ("tiny", "trissm"):
+                line["cpu_baseline"]["c_oracle_1_thread"] = cpu_baseline_c(wl, budget_s=3.0, threads=1)
     print(json.dumps(line))
 
 
@@ -584,11 +586,11 @@ def cpu_baseline(wl, budget_s: float = 12.0):
                                         f"({wl.layers} layer(s)), {el:.1f} s"}
 
 
-def cpu_baseline_c(wl, budget_s: float = 5.0):
+def cpu_baseline_c(wl, budget_s: float = 5.0, threads: int = 0):
     """The C host oracle (oracle/c/, OpenMP over token rows and scan channels,
-    every host core) on the same kind of sample: whole sequences of one layer,
-    repeated until ~budget_s.  None for the workloads it does not cover (the
-    stack, the block form)."""
+    every host core, or `threads` of them) on the same kind of sample: whole
+    sequences of one layer, repeated until ~budget_s.  None for the workloads
+    it does not cover (the stack, the block form)."""
     if wl.layers != 1 or getattr(wl, "block", False):
         return None
     from oracle import c_oracle as C
@@ -596,6 +598,7 @@ def cpu_baseline_c(wl, budget_s: float = 5.0):
     seqs = max(1, min(wl.batch, 4, 1024 // wl.seqlen))
     x, layers = S.make_inputs(wl, seed=0, batch=seqs)
     P = C.Layer(layers[0], wl.act_mode)
+    prev = C.set_threads(threads) if threads > 0 else None
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -604,7 +607,9 @@ def cpu_baseline_c(wl, budget_s: float = 5.0):
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 200:
             break
-    cores = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count() or 1
+    if prev is not None:
+        C.set_threads(prev)
+    cores = threads if threads > 0 else (int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count() or 1)
     return {"value": round(seqs * wl.seqlen * n / el, 1), "unit": UNIT, "cores": cores,
             "kind": "oracle (C, OpenMP)",
             "sample": f"{n} x {seqs} sequences x {wl.seqlen} tokens, {el:.1f} s"}

@@ -9,6 +9,7 @@
 #include "bitssm_oracle.h"
 
 #include <math.h>
+#include <omp.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -336,4 +337,10 @@ int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, in
   }
   free(u); free(delta); free(Bm); free(Cm); free(y); free(A); free(D);
   return bad ? -1 : 0;
+}
+
+int oracle_set_threads(int n) {
+  const int prev = omp_get_max_threads();
+  if (n >= 1) omp_set_num_threads(n);
+  return prev;
 }

@@ -80,6 +80,10 @@ typedef struct oracle_layer {
 int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, int B, int L,
                           int act_mode, const double* h0, double* h_last);
 
+/* Threads the oracle's parallel loops use from now on (n >= 1), for timing
+ * it on one core; returns the previous count. */
+int oracle_set_threads(int n);
+
 #ifdef __cplusplus
 }
 #endif

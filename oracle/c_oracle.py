@@ -29,6 +29,15 @@ _lib.oracle_absmax_codes.argtypes = [_p, ctypes.c_long, _i, _p, _p]
 _lib.oracle_bitlinear_forward.argtypes = [_p, _i, _i, _p, _p, _i, _i, _i, _p]
 _lib.oracle_selective_scan_forward.argtypes = [_p] * 9 + [_i] * 4
 _lib.oracle_bitssm_forward.argtypes = [ctypes.POINTER(oracle_layer), _p, _p, _i, _i, _i, _p, _p]
+_lib.oracle_set_threads.argtypes = [_i]
+_lib.oracle_set_threads.restype = _i
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's parallel loops from now on; returns the previous count."""
+    return _lib.oracle_set_threads(n)
+
+
 for _f in ("oracle_absmean_ternary", "oracle_pack_ternary", "oracle_absmax_codes",
            "oracle_bitlinear_forward", "oracle_selective_scan_forward", "oracle_bitssm_forward"):
     getattr(_lib, _f).restype = _i
