@@ -532,7 +532,7 @@ def run_ours(args):
         "instrumented_ms_per_step": round(main["ev_step_ms"], 5),
         "flush_ms": round(main["flush_ms"], 5),
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the CPU baseline: rank 0 at N = 1 only
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
         c_line = cpu_baseline_c(wl, budget_s=min(5.0, args.cpu_seconds))
         if c_line is not None:
