@@ -227,12 +227,20 @@ static double int_row_codes(const int64_t* acc, int K, double c, int32_t* q, flo
   return m * rms_factor(tmpd, K) / Q_ACT;
 }
 
+static double silu(double v) {
+  const double e = exp(-fabs(v));
+  return v >= 0.0 ? v / (1.0 + e) : v * e / (1.0 + e);
+}
+
 int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, int B, int L,
                           int act_mode, const double* h0, double* h_last) {
   if (!p || !x || !out || B < 0 || L < 0 || (act_mode != 0 && act_mode != 1)) return -1;
   const int d = p->d_model, E = p->d_inner, N = p->d_state, R = p->dt_rank;
   if (d <= 0 || E <= 0 || N <= 0 || R <= 0) return -1;
   if (act_mode == 0 && p->group != 0) return -1;
+  const int block = p->d_conv != 0;
+  if (block && (act_mode != 0 || p->d_conv < 1 || !p->Wq_z || !p->s_z || !p->conv_w || h0))
+    return -1;
   const long T = (long)B * L;
   const int Kmax = (d > E ? d : E);
   double* u = (double*)calloc((size_t)T * E, sizeof(double));
@@ -240,40 +248,95 @@ int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, in
   double* Bm = (double*)calloc((size_t)T * N, sizeof(double));
   double* Cm = (double*)calloc((size_t)T * N, sizeof(double));
   double* y = (double*)calloc((size_t)T * E, sizeof(double));
+  int64_t* acc_in = (int64_t*)calloc((size_t)T * E, sizeof(int64_t));
+  double* deq_x = (double*)calloc((size_t)T, sizeof(double));
+  double* z = block ? (double*)calloc((size_t)T * E, sizeof(double)) : NULL;
+  double* u_pre = block ? (double*)calloc((size_t)T * E, sizeof(double)) : NULL;
   double* A = (double*)malloc(sizeof(double) * E * N);
   double* D = (double*)malloc(sizeof(double) * E);
-  int bad = !u || !delta || !Bm || !Cm || !y || !A || !D;
+  int bad = !u || !delta || !Bm || !Cm || !y || !acc_in || !deq_x || !A || !D ||
+            (block && (!z || !u_pre));
   if (!bad) {
     for (long i = 0; i < (long)E * N; ++i) A[i] = (double)p->A[i];
     for (int e = 0; e < E; ++e) D[e] = (double)p->D[e];
+  }
+  /* phase 1, per token: in_proj (and the gate branch z) */
+  if (!bad) {
 #pragma omp parallel
     {
       int32_t* q = (int32_t*)malloc(sizeof(int32_t) * Kmax);
-      float* tf = (float*)malloc(sizeof(float) * Kmax);
       double* td = (double*)malloc(sizeof(double) * Kmax);
-      int64_t* acc_in = (int64_t*)malloc(sizeof(int64_t) * E);
-      int64_t* acc_x = (int64_t*)malloc(sizeof(int64_t) * (R + 2 * N));
-      double* dt_low = (double*)malloc(sizeof(double) * R);
-      double* draw = (double*)malloc(sizeof(double) * E);
-      if (!q || !tf || !td || !acc_in || !acc_x || !dt_low || !draw) {
+      if (!q || !td) {
 #pragma omp atomic write
         bad = 1;
       } else {
 #pragma omp for schedule(static)
         for (long t = 0; t < T; ++t) {
           const float* xt = x + t * d;
+          for (int k = 0; k < d; ++k) td[k] = (double)xt[k];
           if (act_mode == 0) {
-            /* in_proj on the codes of x */
             const float m = codes_row(xt, d, q);
-            for (int k = 0; k < d; ++k) td[k] = (double)xt[k];
-            const double deq_x = (double)m * rms_factor(td, d) / Q_ACT;
+            deq_x[t] = (double)m * rms_factor(td, d) / Q_ACT;
+            double* dst = block ? u_pre : u;
             for (int e = 0; e < E; ++e) {
-              acc_in[e] = int_dot(q, p->Wq_in + (long)e * d, d);
-              u[t * E + e] = (double)acc_in[e] * (double)p->s_in[0] * deq_x;
+              acc_in[t * E + e] = int_dot(q, p->Wq_in + (long)e * d, d);
+              dst[t * E + e] = (double)acc_in[t * E + e] * (double)p->s_in[0] * deq_x[t];
+              if (block)
+                z[t * E + e] = (double)int_dot(q, p->Wq_z + (long)e * d, d) * (double)p->s_z[0] *
+                               deq_x[t];
             }
-            /* x_proj on the codes of the integer row acc_in */
-            const double c_u = (double)p->s_in[0] * deq_x;
-            const double deq_u = int_row_codes(acc_in, E, c_u, q, tf, td);
+          } else {
+            bl_a16_row(td, d, p->Wq_in, p->s_in, E, p->group, u + t * E);
+          }
+        }
+      }
+      free(q);
+      free(td);
+    }
+  }
+  /* phase 2, block form: u = SiLU(causal depthwise conv of u_pre) */
+  if (!bad && block) {
+    const int K = p->d_conv;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+      for (int e = 0; e < E; ++e)
+        for (int t = 0; t < L; ++t) {
+          double acc = p->conv_b ? (double)p->conv_b[e] : 0.0;
+          for (int k = 0; k < K; ++k) {
+            const int src = t - (K - 1) + k;  /* tap K-1 is the current step */
+            if (src >= 0) acc += (double)p->conv_w[(long)e * K + k] * u_pre[((long)b * L + src) * E + e];
+          }
+          u[((long)b * L + t) * E + e] = silu(acc);
+        }
+  }
+  /* phase 3, per token: x_proj (Delta-down | B | C), Delta-up, softplus */
+  if (!bad) {
+#pragma omp parallel
+    {
+      int32_t* q = (int32_t*)malloc(sizeof(int32_t) * Kmax);
+      float* tf = (float*)malloc(sizeof(float) * Kmax);
+      double* td = (double*)malloc(sizeof(double) * Kmax);
+      int64_t* acc_x = (int64_t*)malloc(sizeof(int64_t) * (R + 2 * N));
+      double* dt_low = (double*)malloc(sizeof(double) * R);
+      double* draw = (double*)malloc(sizeof(double) * E);
+      if (!q || !tf || !td || !acc_x || !dt_low || !draw) {
+#pragma omp atomic write
+        bad = 1;
+      } else {
+#pragma omp for schedule(static)
+        for (long t = 0; t < T; ++t) {
+          if (act_mode == 0) {
+            double deq_u;
+            if (block) {
+              /* codes of the float32 value of u */
+              for (int e = 0; e < E; ++e) tf[e] = (float)u[t * E + e];
+              const float m = codes_row(tf, E, q);
+              deq_u = (double)m * rms_factor(u + t * E, E) / Q_ACT;
+            } else {
+              /* codes of the integer row acc_in */
+              const double c_u = (double)p->s_in[0] * deq_x[t];
+              deq_u = int_row_codes(acc_in + t * E, E, c_u, q, tf, td);
+            }
             for (int j = 0; j < R; ++j) acc_x[j] = int_dot(q, p->Wq_dt_down + (long)j * E, E);
             for (int n = 0; n < N; ++n) {
               acc_x[R + n] = int_dot(q, p->Wq_b + (long)n * E, E);
@@ -290,8 +353,6 @@ int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, in
               delta[t * E + e] = softplus(dr + (double)p->dt_bias[e]);
             }
           } else {
-            for (int k = 0; k < d; ++k) td[k] = (double)xt[k];
-            bl_a16_row(td, d, p->Wq_in, p->s_in, E, p->group, u + t * E);
             bl_a16_row(u + t * E, E, p->Wq_dt_down, p->s_dt_down, R, p->group, dt_low);
             bl_a16_row(u + t * E, E, p->Wq_b, p->s_b, N, p->group, Bm + t * N);
             bl_a16_row(u + t * E, E, p->Wq_c, p->s_c, N, p->group, Cm + t * N);
@@ -301,25 +362,32 @@ int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, in
           }
         }
       }
-      free(q); free(tf); free(td); free(acc_in); free(acc_x); free(dt_low); free(draw);
+      free(q); free(tf); free(td); free(acc_x); free(dt_low); free(draw);
     }
   }
+  /* phase 4: the scan */
   if (!bad)
     bad = oracle_selective_scan_forward(u, delta, A, Bm, Cm, D, h0, y, h_last, B, L, E, N) != 0;
+  /* phase 5, per token: (gate and) out_proj */
   if (!bad) {
 #pragma omp parallel
     {
       int32_t* q = (int32_t*)malloc(sizeof(int32_t) * E);
       float* tf = (float*)malloc(sizeof(float) * E);
-      if (!q || !tf) {
+      double* yg = (double*)malloc(sizeof(double) * E);
+      if (!q || !tf || !yg) {
 #pragma omp atomic write
         bad = 1;
       } else {
 #pragma omp for schedule(static)
         for (long t = 0; t < T; ++t) {
           const double* yt = y + t * E;
+          if (block) {
+            for (int e = 0; e < E; ++e) yg[e] = yt[e] * silu(z[t * E + e]);
+            yt = yg;
+          }
           if (act_mode == 0) {
-            /* out_proj on the codes of the float32 value of y */
+            /* out_proj on the codes of the float32 value of y (or y_g) */
             for (int e = 0; e < E; ++e) tf[e] = (float)yt[e];
             const float m = codes_row(tf, E, q);
             const double deq_y = (double)m * rms_factor(yt, E) / Q_ACT;
@@ -331,11 +399,55 @@ int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, in
           }
         }
       }
-      free(q);
-      free(tf);
+      free(q); free(tf); free(yg);
     }
   }
-  free(u); free(delta); free(Bm); free(Cm); free(y); free(A); free(D);
+  free(u); free(delta); free(Bm); free(Cm); free(y); free(acc_in); free(deq_x); free(z);
+  free(u_pre); free(A); free(D);
+  return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------ SSD scan */
+
+int oracle_ssd_scan_forward(const double* x, const double* dt, const double* A, const double* Bm,
+                            const double* Cm, const double* D, const double* S0, double* y,
+                            double* S_last, int B, int L, int H, int P, int G, int N) {
+  if (B < 0 || L < 0 || H <= 0 || P <= 0 || G <= 0 || N <= 0 || H % G != 0 || !A) return -1;
+  if (L > 0 && (!x || !dt || !Bm || !Cm || !y)) return -1;
+  const int per = H / G;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* S = (double*)malloc(sizeof(double) * N);
+    if (!S) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+#pragma omp for collapse(3) schedule(static)
+      for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+          for (int pp = 0; pp < P; ++pp) {
+            const int g = h / per;
+            const long srow = (((long)b * H + h) * P + pp) * N;
+            for (int n = 0; n < N; ++n) S[n] = S0 ? S0[srow + n] : 0.0;
+            for (int t = 0; t < L; ++t) {
+              const double dtv = dt[((long)b * L + t) * H + h];
+              const double a = exp(dtv * A[h]);
+              const double xv = x[(((long)b * L + t) * H + h) * P + pp];
+              const long bc = (((long)b * L + t) * G + g) * N;
+              double acc = 0.0;
+              for (int n = 0; n < N; ++n) {
+                S[n] = a * S[n] + dtv * xv * Bm[bc + n];
+                acc += S[n] * Cm[bc + n];
+              }
+              y[(((long)b * L + t) * H + h) * P + pp] = acc + (D ? D[h] : 0.0) * xv;
+            }
+            if (S_last)
+              for (int n = 0; n < N; ++n) S_last[srow + n] = S[n];
+          }
+    }
+    free(S);
+  }
   return bad ? -1 : 0;
 }
 

@@ -70,6 +70,13 @@ typedef struct oracle_layer {
   const float *s_in, *s_dt_down, *s_b, *s_c, *s_dt_up, *s_out;
   const float *A, *D, *dt_bias;
   int d_model, d_inner, d_state, dt_rank, group;
+  /* Mamba-1 block form (d_conv != 0, A8, zero start state only): the gate
+   * branch z_proj [E, d] and the depthwise causal conv taps [E, d_conv]
+   * (tap d_conv-1 on the current step) and bias [E] (may be NULL). */
+  const int8_t* Wq_z;
+  const float* s_z;
+  const float *conv_w, *conv_b;
+  int d_conv;
 } oracle_layer;
 
 /* The mixer on x [B, L, d_model] (float32 values) -> out double [B, L, d].
@@ -79,6 +86,15 @@ typedef struct oracle_layer {
  * h0 / h_last as in oracle_selective_scan_forward (nullable). */
 int oracle_bitssm_forward(const oracle_layer* p, const float* x, double* out, int B, int L,
                           int act_mode, const double* h0, double* h_last);
+
+/* SSD scan of Mamba-2 in float64, step by step: x, y [B, L, H, P];
+ * dt [B, L, H] (after the softplus); A [H]; Bm, Cm [B, L, G, N]; D [H] or
+ * NULL; S0, S_last [B, H, P, N] or NULL; head h reads group h / (H / G).
+ *   S_t = exp(dt_t[h] A[h]) S_{t-1} + dt_t[h] x_t[h] (outer) B_t[g]
+ *   y_t[h] = S_t C_t[g] + D[h] x_t[h] */
+int oracle_ssd_scan_forward(const double* x, const double* dt, const double* A, const double* Bm,
+                            const double* Cm, const double* D, const double* S0, double* y,
+                            double* S_last, int B, int L, int H, int P, int G, int N);
 
 /* Threads the oracle's parallel loops use from now on (n >= 1), for timing
  * it on one core; returns the previous count. */

@@ -20,7 +20,8 @@ class oracle_layer(ctypes.Structure):
     _fields_ = [(n, _p) for n in ("Wq_in", "Wq_dt_down", "Wq_b", "Wq_c", "Wq_dt_up", "Wq_out",
                                   "s_in", "s_dt_down", "s_b", "s_c", "s_dt_up", "s_out",
                                   "A", "D", "dt_bias")] + \
-               [(n, _i) for n in ("d_model", "d_inner", "d_state", "dt_rank", "group")]
+               [(n, _i) for n in ("d_model", "d_inner", "d_state", "dt_rank", "group")] + \
+               [("Wq_z", _p), ("s_z", _p), ("conv_w", _p), ("conv_b", _p), ("d_conv", _i)]
 
 
 _lib.oracle_absmean_ternary.argtypes = [_p, _i, _i, _i, _p, _p]
@@ -29,6 +30,8 @@ _lib.oracle_absmax_codes.argtypes = [_p, ctypes.c_long, _i, _p, _p]
 _lib.oracle_bitlinear_forward.argtypes = [_p, _i, _i, _p, _p, _i, _i, _i, _p]
 _lib.oracle_selective_scan_forward.argtypes = [_p] * 9 + [_i] * 4
 _lib.oracle_bitssm_forward.argtypes = [ctypes.POINTER(oracle_layer), _p, _p, _i, _i, _i, _p, _p]
+_lib.oracle_ssd_scan_forward.argtypes = [_p] * 9 + [_i] * 6
+_lib.oracle_ssd_scan_forward.restype = _i
 _lib.oracle_set_threads.argtypes = [_i]
 _lib.oracle_set_threads.restype = _i
 
@@ -126,6 +129,16 @@ class Layer:
                               _ptr(self.keep["dt_bias"]),
                               lw.W_in.shape[1], lw.W_in.shape[0], lw.A.shape[1],
                               lw.W_dt_down.shape[0], self.group)
+        if getattr(lw, "W_z", None) is not None:  # Mamba-1 block form
+            self.keep["W_z"] = absmean_ternary(lw.W_z, self.group)
+            self.keep["s_z"] = _c(np.atleast_1d(self.keep["W_z"][1]), np.float32)
+            self.keep["conv_w"] = _c(lw.conv_w, np.float32)
+            self.keep["conv_b"] = _c(lw.conv_b, np.float32)
+            self.c.Wq_z = _ptr(self.keep["W_z"][0])
+            self.c.s_z = _ptr(self.keep["s_z"])
+            self.c.conv_w = _ptr(self.keep["conv_w"])
+            self.c.conv_b = _ptr(self.keep["conv_b"])
+            self.c.d_conv = lw.conv_w.shape[1]
 
 
 def bitssm_forward(x, layer: Layer, h0=None):
@@ -138,3 +151,17 @@ def bitssm_forward(x, layer: Layer, h0=None):
     _ok(_lib.oracle_bitssm_forward(ctypes.byref(layer.c), _ptr(x), _ptr(out), Bsz, L,
                                    layer.act_mode, _ptr(h0), _ptr(h)), "bitssm_forward")
     return out, h
+
+
+def ssd_scan(x, dt, A, Bm, Cm, D, S0=None):
+    x, dt, A, Bm, Cm, D = (_c(a, np.float64) for a in (x, dt, A, Bm, Cm, D))
+    Bsz, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    S0 = None if S0 is None else _c(S0, np.float64)
+    y = np.zeros_like(x)
+    S = np.zeros((Bsz, H, P, N))
+    _ok(_lib.oracle_ssd_scan_forward(_ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(D),
+                                     _ptr(S0), _ptr(y), _ptr(S), Bsz, L, H, P, G, N),
+        "ssd_scan_forward")
+    return y, S
+

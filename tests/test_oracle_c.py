@@ -13,6 +13,7 @@ import pytest
 
 from oracle import bitssm_oracle as O
 from oracle import c_oracle as C
+from oracle import ssd_oracle as SSD
 from ternary_weight_selective_b200 import synthetic as S
 from tests._helpers import rel_err
 
@@ -103,3 +104,26 @@ def test_invalid_arguments_are_refused():
         C.bitlinear(np.zeros((2, 8), np.float32), np.zeros((4, 8), np.int8), np.ones(1), 128, 0)
     with pytest.raises(ValueError):
         C.absmean_ternary(np.zeros((0, 4), np.float32))
+
+
+@pytest.mark.parametrize("K,B,L", [(4, 2, 30), (2, 1, 3), (3, 2, 1)])
+def test_block_form_matches_numpy(K, B, L):
+    wl = S.Workload("blk_c", B, L, 64, 128, 16, 4, "f32", "A8", block=True, d_conv=K)
+    x, layers = S.make_inputs(wl, seed=K * 10 + L)
+    out_c, h_c = C.bitssm_forward(x, C.Layer(layers[0], "A8"))
+    out_n, st = O.bitssm_block_a8(x, O.TernaryLayer(layers[0], "A8"))
+    assert rel_err(out_c, out_n) <= 1e-12
+    assert rel_err(h_c, st["h_last"]) <= 1e-12
+    # the block form has no carried-state form
+    with pytest.raises(ValueError):
+        C.bitssm_forward(x, C.Layer(layers[0], "A8"), np.zeros((B, 128, 16)))
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_ssd_scan_matches_numpy(G):
+    args = S.random_ssd_inputs(G, 2, 21, 4, 8, G, 16)
+    S0 = np.random.default_rng(2).normal(size=(2, 4, 8, 16))
+    y_c, s_c = C.ssd_scan(*args, S0=S0)
+    y_n, s_n = SSD.ssd_sequential(*args, S0=S0)
+    assert rel_err(y_c, y_n) <= 1e-12 and rel_err(s_c, s_n) <= 1e-12
+
