@@ -164,6 +164,16 @@ int bitssm_pack_workspace_size(int n_out, int k_in, int group, size_t* bytes);
 int bitssm_pack_ternary(const float* W, int n_out, int k_in, int group, uint8_t* packed,
                         float* scales, void* ws, size_t ws_bytes, void* stream);
 
+/* Host-side check of a packed ternary matrix held in HOST memory (for
+ * weights that come from a file rather than from bitssm_pack_ternary):
+ * packed uint8 [n_out, ceil(k_in/4)] in the 2-bit encoding above.  Counts
+ * the elements of the matrix that hold the invalid code 3 into *bad (the
+ * padding elements past k_in must hold code 1 and are counted too when they
+ * do not).  Returns BITSSM_OK when *bad == 0, BITSSM_ERR_INVALID_ARG when
+ * any code is invalid or an argument is.  No device work.  The pages give no
+ * interface for this; the encoding is the one packing defines. */
+int bitssm_check_packed(const uint8_t* packed_host, int n_out, int k_in, long* bad);
+
 /* ---------------------------------------------------------------------
  * BitLinear forward on M input rows (TriSSM README: opening paragraph and
  * the caption "an RMSNorm precedes each ternary projection"; multiply-free

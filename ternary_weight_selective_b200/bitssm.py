@@ -99,6 +99,7 @@ _SIGS = {
     "bitssm_forward_launches": (_i, [_P_LAYER, _i, _i, _i]),
     "bitssm_selftest_wait": (_i, [ctypes.c_uint, _vp]),
     "ssd_scan_forward": (_i, [_vp] * 9 + [_i] * 6 + [_vp]),
+    "bitssm_check_packed": (_i, [_vp, _i, _i, ctypes.POINTER(ctypes.c_long)]),
     "bitssm_forward_timed": (_i, [_P_LAYER, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _sz,
                                   ctypes.POINTER(_vp), _i, _vp]),
     "bitssm_prepared_size": (_i, [_P_LAYER, _i, ctypes.POINTER(_sz)]),
@@ -227,6 +228,17 @@ def bitssm_step(layer: bitssm_layer, x, out, residual, h, B, dtype, act_mode, ws
     _check(_lib.bitssm_step(ctypes.byref(layer), _ptr(x), _ptr(out), _ptr(residual), _ptr(h), B,
                             dtype, act_mode, _ptr(ws), ws_bytes, _stream(stream)),
            "bitssm_step")
+
+
+def bitssm_check_packed(packed_host, n_out: int, k_in: int) -> int:
+    """Number of invalid codes in a packed matrix in host memory (a numpy
+    uint8 array or an address); 0 when the matrix is valid."""
+    bad = ctypes.c_long(0)
+    addr = packed_host if isinstance(packed_host, int) else packed_host.ctypes.data
+    rc = _lib.bitssm_check_packed(addr, n_out, k_in, ctypes.byref(bad))
+    if rc not in (OK, ERR_INVALID_ARG) or (rc == ERR_INVALID_ARG and bad.value == 0):
+        _check(rc, "bitssm_check_packed")
+    return bad.value
 
 
 def ssd_scan_forward(x, dt, A, Bm, Cm, D, S0, y, S_last, B, L, H, P, G, N, stream=None):

@@ -1104,6 +1104,24 @@ int bitssm_pack_ternary(const float* W, int n_out, int k_in, int group, uint8_t*
   return launch_status();
 }
 
+int bitssm_check_packed(const uint8_t* packed_host, int n_out, int k_in, long* bad) {
+  if (packed_host == nullptr || bad == nullptr || n_out <= 0 || k_in <= 0)
+    return BITSSM_ERR_INVALID_ARG;
+  const int kb = (k_in + 3) / 4;
+  long count = 0;
+  for (long n = 0; n < n_out; ++n)
+    for (int b = 0; b < kb; ++b) {
+      const unsigned byte = packed_host[n * kb + b];
+      for (int i = 0; i < 4; ++i) {
+        const unsigned code = (byte >> (2 * i)) & 3u;
+        const bool pad = 4 * b + i >= k_in;
+        if (code == 3u || (pad && code != 1u)) ++count;
+      }
+    }
+  *bad = count;
+  return count == 0 ? BITSSM_OK : BITSSM_ERR_INVALID_ARG;
+}
+
 // ---------------------------------------------------------------- BitLinear
 int bitlinear_workspace_size(const bitssm_tw* w, int M, int act_mode, size_t* bytes) {
   if (bytes == nullptr || !tw_ok(w) || M < 0) return BITSSM_ERR_INVALID_ARG;
