@@ -46,7 +46,7 @@ extern "C" {
 enum bitssm_status_code {
   BITSSM_OK = 0,
   BITSSM_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad enum */
-  BITSSM_ERR_UNSUPPORTED_SHAPE = 2,/* a size this build does not support */
+  BITSSM_ERR_UNSUPPORTED_SHAPE = 2,/* a size the library does not support */
   BITSSM_ERR_WORKSPACE = 3,        /* workspace missing, misaligned or too small */
   BITSSM_ERR_CUDA = 4,             /* a CUDA launch or runtime call failed */
   BITSSM_ERR_TIMEOUT = 5,          /* a bounded device wait ran out (device error word) */
