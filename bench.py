@@ -189,6 +189,37 @@ def layer_bytes_per_token(wl):
     return pre_bytes_per_token(wl) + scan_bytes_per_token(E, N, Rp) + post_bytes_per_token(wl)
 
 
+def named_roofline(wl, names, kernel_ms, peaks, peak_kind):
+    """The projections against the tensor pipe of their operand type: the
+    GEMM operations per token (2 (d E + E (R + 2N) + E d) on the tensor core;
+    Delta-up runs as a dot product in the A8 fused scan, or as a GEMM) over
+    the summed times of the kernels that run them, against the measured bf16
+    burst peak (x 2 for int8: the nominal dense int8 / bf16 ratio).  The
+    scan's HBM fraction is in the roofline object."""
+    d, E, N, R = wl.d_model, wl.d_inner, wl.d_state, wl.dt_rank
+    gemm_kernels = [i for i, n in enumerate(names)
+                    if n.startswith(("bitssm_pre", "bitssm_post", "gemm_"))]
+    if not gemm_kernels:
+        return None
+    fused_dt_up = any(n == "selective_scan_fused_dt" for n in names)
+    ops = 2 * (d * E + E * (R + 2 * N) + E * d) + (0 if fused_dt_up else 2 * R * E)
+    if getattr(wl, "block", False):
+        ops += 2 * d * E                       # z_proj
+    t_s = sum(kernel_ms[i] for i in gemm_kernels) / 1e3
+    if t_s <= 0:
+        return None
+    int8 = wl.act_mode == "A8"
+    peak = peaks["bf16_tflops"] * (2.0 if int8 else 1.0)
+    achieved = ops * wl.tokens / t_s / 1e12
+    return {"projections": [names[i] for i in gemm_kernels],
+            "unit": "TOPS" if int8 else "TFLOP/s", "achieved": round(achieved, 2),
+            "peak": round(peak, 1), "frac": round(achieved / peak, 4),
+            "ops_per_token": ops,
+            "peak_source": f"{peak_kind} bf16_tflops" + (" x 2 (int8 / bf16 nominal ratio)" if int8 else ""),
+            "note": "the kernel times include the fused quantisers and epilogues; "
+                    "at d = 256 these kernels are HBM-bound (see roofline)"}
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -519,6 +550,7 @@ def run_ours(args):
         "weights": "expanded once before the timed region (bitssm_prepare_weights)",
         "value_with_per_call_weight_expansion": round(T * world / (unprep["ms"] / 1e3), 1),
         "layer_hbm_gbs_algorithmic": round(layer_gbs, 1),
+        "named_roofline_projections": named_roofline(wl, names, avg_kernel_ms, peaks, peak_kind),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": io_bytes,
                 "d2h_bytes_per_step": io_bytes, "steps": n_e2e,
                 "pipelining": "serving loop: step k+1's H2D and step k-1's D2H (own streams, "
