@@ -348,10 +348,11 @@ def run_ours(args):
         torch.cuda.synchronize()
         t_wall = time.perf_counter()
         plain_ms = flush_ms = 0.0
-        for _ in range(R):
-            plain_ms += replay_ms(g_plain)
-            flush_ms += replay_ms(g_flush)
-        torch.cuda.synchronize()
+        with torch.cuda.nvtx.range("bitssm timed region"):
+            for _ in range(R):
+                plain_ms += replay_ms(g_plain)
+                flush_ms += replay_ms(g_flush)
+            torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
         if world > 1:
             dist.barrier()
@@ -359,8 +360,9 @@ def run_ours(args):
         kern_ms = [[0.0] * nl for _ in range(n_layers)]
         ev_step_ms = 0.0
         for _ in range(R):
-            g_ev.replay()
-            torch.cuda.synchronize()
+            with torch.cuda.nvtx.range("bitssm per-kernel events"):
+                g_ev.replay()
+                torch.cuda.synchronize()
             for evs in gevents:
                 for li in range(n_layers):
                     e = evs[li * (nl + 1):(li + 1) * (nl + 1)]
@@ -446,7 +448,8 @@ def run_ours(args):
         dist.barrier()
     ea2, eb2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea2.record(comp)
-    e2e_run(n_e2e)
+    with torch.cuda.nvtx.range("bitssm end-to-end serving loop"):
+        e2e_run(n_e2e)
     eb2.record(comp)
     torch.cuda.synchronize()
     e2e_ms = ea2.elapsed_time(eb2)
@@ -777,9 +780,10 @@ def run_ssd(args):
     time.sleep(0.3)
     torch.cuda.synchronize()
     plain = fl = 0.0
-    for _ in range(R):
-        plain += replay_ms(g_plain)
-        fl += replay_ms(g_flush)
+    with torch.cuda.nvtx.range("ssd timed region"):
+        for _ in range(R):
+            plain += replay_ms(g_plain)
+            fl += replay_ms(g_flush)
     clocks = sampler.stop()
     K = Gr * R
     ms = (plain - fl) / K
