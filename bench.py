@@ -656,7 +656,9 @@ def run_reference(args):
         return
     from ternary_weight_selective_b200 import synthetic as S
     wl = S.WORKLOADS[args.workload]
-    seqs = max(1, min(wl.batch, 2))
+    # each step is a bounded sample of the workload: two whole sequences, or
+    # one when many steps are asked for, so the run stays within minutes
+    seqs = max(1, min(wl.batch, 2 if args.steps + args.warmup <= 1000 else 1))
     run, tokens = oracle_sample(wl, seqs)
     for _ in range(args.warmup):
         run()
